@@ -1,0 +1,187 @@
+/*
+ * Plain, slow, fp64 CPU oracle for paged decode attention and the slot-mapped
+ * KV write.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * bench's CPU-baseline leg call it; the product path never does.  It shares
+ * no code, header or helper with the CUDA library.
+ *
+ * Sources (web pages on vLLM / PagedAttention):
+ *  [P3] "4. vLLM核心机制：PagedAttention、Continuous Batching、动态批处理",
+ *       section 4.2: the KV cache is cut into fixed-size pages of 16 or 32
+ *       tokens; a per-request page table maps logical page i to a physical
+ *       page anywhere in the pool (worked example: logical 0,1,2 -> physical
+ *       7,2,5); attention looks the pages up one by one through the table and
+ *       never assumes the K/V rows are contiguous; pages of a shared prefix
+ *       may be named by several requests' tables.
+ *       Section 4.3: each decode iteration produces the new token together
+ *       with the updated KV cache.
+ *  [P1] "vLLM：大型语言模型推理优化的革命性突破", section 2.1: the attention
+ *       kernel indexes the scattered blocks through the table with no data
+ *       movement and no zero padding, i.e. the result is ordinary attention
+ *       over the logical sequence.
+ *  [P2] pinggu.org forum post, section "PagedAttention：让显存像虚拟内存一样灵活":
+ *       a page holds a fixed number of tokens (16 by default) and logical
+ *       continuity is separated from physical placement.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *  - cache layout [num_blocks][num_kv_heads][block_size][head_dim];
+ *  - query head hq reads kv head hq / (num_q_heads / num_kv_heads);
+ *  - context_lens[s] counts every token the step attends to, including the
+ *    one written by this step's KV write;
+ *  - a negative slot in the slot mapping means "write nothing";
+ *  - a sequence with context length 0 yields an all-zero output row.
+ *
+ * Storage elements are IEEE binary16 (dtype 1) or bfloat16 (dtype 2) bit
+ * patterns; they are widened to double here from their format definitions.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG -1
+#define ORACLE_ERR_BLOCK_ID -2
+#define ORACLE_ERR_SLOT -3
+#define ORACLE_ERR_CONTEXT -4
+#define ORACLE_ERR_NOMEM -5
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double oracle_half_to_double(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double mag;
+    if (e == 0) {
+        mag = ldexp((double)f, -24); /* subnormal: f * 2^-14 * 2^-10 */
+    } else if (e == 31) {
+        mag = f ? NAN : INFINITY;
+    } else {
+        mag = ldexp((double)(f + 1024), e - 25); /* (1 + f/1024) * 2^(e-15) */
+    }
+    return sign ? -mag : mag;
+}
+
+/* bfloat16: the upper 16 bits of an IEEE binary32. */
+double oracle_bf16_to_double(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float x;
+    memcpy(&x, &u, sizeof x);
+    return (double)x;
+}
+
+static double widen(uint16_t bits, int dtype) {
+    return dtype == 2 ? oracle_bf16_to_double(bits) : oracle_half_to_double(bits);
+}
+
+/*
+ * KV write ([P3] section 4.3): for every new token t and kv head h, the
+ * slot s = slot_mapping[t] names physical block s / block_size and row
+ * s % block_size; k[t][h][:] and v[t][h][:] are copied there bit for bit.
+ * k, v: [num_tokens][num_kv_heads][head_dim]; caches as in the layout above.
+ */
+int oracle_write_kv(const uint16_t *k, const uint16_t *v, uint16_t *k_cache, uint16_t *v_cache,
+                    const int64_t *slot_mapping, int64_t num_tokens, int64_t num_kv_heads,
+                    int64_t head_dim, int64_t block_size, int64_t num_blocks) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0)
+        return ORACLE_ERR_ARG;
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * block_size) return ORACLE_ERR_SLOT;
+        int64_t block = slot / block_size;
+        int64_t row = slot % block_size;
+        for (int64_t h = 0; h < num_kv_heads; ++h) {
+            for (int64_t i = 0; i < head_dim; ++i) {
+                int64_t src = (t * num_kv_heads + h) * head_dim + i;
+                int64_t dst = ((block * num_kv_heads + h) * block_size + row) * head_dim + i;
+                k_cache[dst] = k[src];
+                v_cache[dst] = v[src];
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Decode attention for one new query token per sequence.  For sequence s and
+ * query head hq (kv head h):
+ *   1. gather the L = context_lens[s] logical tokens through the page table:
+ *      token j lives in physical block block_tables[s][j / block_size], row
+ *      j % block_size ([P3] section 4.2), giving contiguous K[L][d], V[L][d];
+ *   2. z_j = scale * sum_i q[i] * K[j][i];
+ *   3. w_j = exp(z_j - max_j z_j),  Z = sum_j w_j;
+ *   4. out[i] = sum_j (w_j / Z) * V[j][i]                    ([P1] section 2.1)
+ * q: [num_seqs][num_q_heads][head_dim]; block_tables: [num_seqs][table_stride];
+ * out: [num_seqs][num_q_heads][head_dim] doubles.
+ */
+int oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                  const int32_t *block_tables, int64_t table_stride, const int32_t *context_lens,
+                  int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                  int64_t block_size, int64_t num_blocks, int dtype, double scale, double *out) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_q_heads % num_kv_heads != 0 || (dtype != 1 && dtype != 2))
+        return ORACLE_ERR_ARG;
+    int64_t group = num_q_heads / num_kv_heads;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t L = context_lens[s];
+        if (L < 0 || L > table_stride * block_size) return ORACLE_ERR_CONTEXT;
+        for (int64_t j = 0; j < L; j += block_size) {
+            int32_t p = block_tables[s * table_stride + j / block_size];
+            if (p < 0 || p >= num_blocks) return ORACLE_ERR_BLOCK_ID;
+        }
+    }
+    double *K = NULL, *V = NULL, *z = NULL;
+    int rc = ORACLE_OK;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t L = context_lens[s];
+        if (L > 0) {
+            K = (double *)malloc((size_t)(L * head_dim) * sizeof(double));
+            V = (double *)malloc((size_t)(L * head_dim) * sizeof(double));
+            z = (double *)malloc((size_t)L * sizeof(double));
+            if (!K || !V || !z) { rc = ORACLE_ERR_NOMEM; goto done; }
+        }
+        for (int64_t hq = 0; hq < num_q_heads; ++hq) {
+            int64_t h = hq / group;
+            double *o = out + (s * num_q_heads + hq) * head_dim;
+            for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;
+            if (L == 0) continue;
+            /* step 1: gather */
+            for (int64_t j = 0; j < L; ++j) {
+                int64_t p = block_tables[s * table_stride + j / block_size];
+                int64_t row = j % block_size;
+                const uint16_t *kr = k_cache + ((p * num_kv_heads + h) * block_size + row) * head_dim;
+                const uint16_t *vr = v_cache + ((p * num_kv_heads + h) * block_size + row) * head_dim;
+                for (int64_t i = 0; i < head_dim; ++i) {
+                    K[j * head_dim + i] = widen(kr[i], dtype);
+                    V[j * head_dim + i] = widen(vr[i], dtype);
+                }
+            }
+            /* step 2: scaled dot products */
+            const uint16_t *qr = q + (s * num_q_heads + hq) * head_dim;
+            for (int64_t j = 0; j < L; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < head_dim; ++i) acc += widen(qr[i], dtype) * K[j * head_dim + i];
+                z[j] = scale * acc;
+            }
+            /* step 3: softmax weights */
+            double m = z[0];
+            for (int64_t j = 1; j < L; ++j)
+                if (z[j] > m) m = z[j];
+            double Z = 0.0;
+            for (int64_t j = 0; j < L; ++j) {
+                z[j] = exp(z[j] - m);
+                Z += z[j];
+            }
+            /* step 4: weighted sum of V rows */
+            for (int64_t j = 0; j < L; ++j) {
+                double w = z[j] / Z;
+                for (int64_t i = 0; i < head_dim; ++i) o[i] += w * V[j * head_dim + i];
+            }
+        }
+        free(K); free(V); free(z);
+        K = V = z = NULL;
+    }
+done:
+    free(K); free(V); free(z);
+    return rc;
+}

@@ -1,0 +1,91 @@
+"""Plant plausible mistakes in a copy of the C oracle and check that the pins catch each one.
+
+Every mutant is one textual edit of ``oracle/pa_oracle.c`` (a wrong index, a
+dropped term, a flipped sign, swapped operands), compiled into a temporary
+library on the CPU.  A mutant that no pin rejects would mean the pins leave
+that part of the oracle unchecked.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
+
+MUTANTS = {
+    "row_uses_division": ("int64_t row = j % block_size;", "int64_t row = j / block_size;"),
+    "table_uses_modulo": ("block_tables[s * table_stride + j / block_size];\n                int64_t row",
+                          "block_tables[s * table_stride + j % block_size];\n                int64_t row"),
+    "gqa_modulo_grouping": ("int64_t h = hq / group;", "int64_t h = hq % num_kv_heads;"),
+    "dropped_scale": ("z[j] = scale * acc;", "z[j] = acc;"),
+    "softmax_sign": ("z[j] = exp(z[j] - m);", "z[j] = exp(m - z[j]);"),
+    "no_max_shift": ("z[j] = exp(z[j] - m);", "z[j] = exp(z[j]);"),
+    "dropped_normaliser": ("double w = z[j] / Z;", "double w = z[j];"),
+    "k_v_swapped": ("K[j * head_dim + i] = widen(kr[i], dtype);", "K[j * head_dim + i] = widen(vr[i], dtype);"),
+    "query_of_kv_head": ("q + (s * num_q_heads + hq) * head_dim;", "q + (s * num_q_heads + h) * head_dim;"),
+    "last_token_dropped": ("for (int64_t j = 0; j < L; ++j) {\n                int64_t p",
+                           "for (int64_t j = 0; j < L - 1; ++j) {\n                int64_t p"),
+    "fp16_no_implicit_bit": ("ldexp((double)(f + 1024), e - 25)", "ldexp((double)f, e - 25)"),
+    "fp16_bias_off_by_one": ("ldexp((double)(f + 1024), e - 25)", "ldexp((double)(f + 1024), e - 24)"),
+    "fp16_subnormal_scale": ("ldexp((double)f, -24);", "ldexp((double)f, -25);"),
+    "bf16_shift": ("((uint32_t)b) << 16;", "((uint32_t)b) << 15;"),
+    "dtype_swapped": ("return dtype == 2 ? oracle_bf16_to_double(bits)", "return dtype == 1 ? oracle_bf16_to_double(bits)"),
+    "write_row_division": ("int64_t row = slot % block_size;", "int64_t row = slot / block_size % block_size;"),
+    "write_k_from_v": ("k_cache[dst] = k[src];", "k_cache[dst] = v[src];"),
+    "write_head_stride": ("int64_t dst = ((block * num_kv_heads + h) * block_size + row) * head_dim + i;",
+                          "int64_t dst = ((block * num_kv_heads) * block_size + row) * head_dim + i;"),
+    "write_negative_slots": ("if (slot < 0) continue;", "if (slot < 0) slot = 0;"),
+    "zero_length_garbage": ("for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;\n            if (L == 0) continue;",
+                            "if (L == 0) { o[0] = 1.0; continue; }\n            for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;"),
+}
+
+
+_RUNNER = """
+import json, sys
+sys.path[:0] = sys.argv[2:]
+from oracle_pins import ALL_PINS
+failed = []
+for pin in ALL_PINS:
+    try:
+        pin(sys.argv[1])
+    except (AssertionError, ValueError):
+        failed.append(pin.__name__)
+print(json.dumps(failed))
+"""
+
+
+def _failing_pins(lib_path):
+    """Run every pin against ``lib_path`` in a child process (a mutant may read out of bounds)."""
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    res = subprocess.run([sys.executable, "-c", _RUNNER, lib_path, here, root], capture_output=True, text=True,
+                         timeout=600)
+    if res.returncode < 0:
+        return [f"crashed (signal {-res.returncode})"]
+    assert res.returncode == 0, f"pin runner failed: {res.stderr[-2000:]}"
+    return json.loads(res.stdout.strip().splitlines()[-1])
+
+
+def test_runner_accepts_the_real_oracle(tmp_path):
+    """Control: the unmodified source, built the same way, passes every pin in the runner."""
+    lib = str(tmp_path / "libpa_oracle_control.so")
+    oracle.build(SRC, lib)
+    assert _failing_pins(lib) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mutated = tmp_path / "pa_oracle_mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = str(tmp_path / "libpa_oracle_mutant.so")
+    oracle.build(str(mutated), lib)
+    failed = _failing_pins(lib)
+    assert failed, f"mutant {name} passes every pin"
+    print(f"{name}: caught by {failed}")
