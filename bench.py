@@ -1,0 +1,376 @@
+"""Benchmark of the paged decode step on B200: KV GB/s (fraction of HBM peak) and seq-steps/s.
+
+One step = ``pa_write_kv`` of each sequence's new token, then ``pa_decode`` over
+the block-paged cache (all kernels of the hot path), on seeded synthetic data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+N > 1 is launched by torchrun (one rank per GPU): each rank owns an independent
+batch of the same shape (weak scaling, no data-path collective); timing is the
+max over ranks.  ``--impl reference`` times the fp64 CPU oracle on host cores
+on a bounded sample of the same workload.  Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s (fraction of HBM peak) and seq-steps/s, 1×B200"
+DEFAULT_WORKLOAD = "llama2_7b_decode"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+SEEDS = {"tiny_decode": 1, "llama2_7b_decode": 2, "gqa_llama3_decode": 3, "long_context_splitk": 4,
+         "shared_prefix_step": 5}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.NAMED))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def make_workload(name: str, rank: int):
+    return W.NAMED[name](seed=SEEDS[name] + 1000 * rank)
+
+
+def step_bytes(wl, st):
+    """Algorithmic bytes of one decode call: K and V of exactly the live tokens, q, out,
+    the table entries read and the lengths (partial-block slack not counted)."""
+    elem = 2
+    kv = W.kv_bytes(st, wl.num_kv_heads, wl.head_dim, elem)
+    qo = 2 * st.num_seqs * wl.num_q_heads * wl.head_dim * elem
+    nblk = int(sum(-(-int(L) // wl.block_size) for L in st.context_lens))
+    return kv, kv + qo + 4 * nblk + 4 * st.num_seqs
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) in a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = repr(e)
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self.nvml
+        get_reasons = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            n.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(), n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM),
+                                     int(get_reasons(self.h))))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"error": self.err}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = inside if len(inside) >= 3 else self.samples
+        if not use:
+            return {"error": "no samples"}
+        mask = 0
+        for s in use:
+            mask |= s[2]
+        return {"sm_mhz": statistics.median(s[1] for s in use), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(k for k, v in self.REASONS.items() if mask & v and k != "gpu_idle"),
+                "samples": len(use), "window": "timed region" if use is inside else "whole run"}
+
+
+def cpu_oracle_rate(wl, st, seconds: float):
+    """Times the fp64 C oracle (single thread) on the first sequences of the step, about
+    ``seconds`` of work; returns (GB/s of KV it processed, description)."""
+    import oracle
+    kc, vc = oracle.write_kv(st.k_new, st.v_new, wl.k_cache, wl.v_cache, st.slot_mapping, wl.block_size)
+    order = np.arange(st.num_seqs)
+    done_bytes, elapsed, n = 0, 0.0, 0
+    per_seq = wl.num_kv_heads * wl.head_dim * 2 * 2
+    while elapsed < seconds and n < st.num_seqs:
+        s = order[n:n + 1]
+        t = time.perf_counter()
+        oracle.decode(st.q[s], kc, vc, st.block_tables[s], st.context_lens[s], wl.scale, wl.dtype)
+        elapsed += time.perf_counter() - t
+        done_bytes += int(st.context_lens[s].sum()) * per_seq
+        n += 1
+    return done_bytes / elapsed / 1e9, n, elapsed
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = make_workload(args.workload, 0)
+    st = wl.steps[0]
+    import oracle
+    kc, vc = oracle.write_kv(st.k_new, st.v_new, wl.k_cache, wl.v_cache, st.slot_mapping, wl.block_size)
+    per_seq = wl.num_kv_heads * wl.head_dim * 2 * 2
+    # one step = the oracle on a 2-sequence sample of the batch (rotating), bounded work per step
+    sample = 2
+    times, nbytes = [], []
+    for i in range(args.warmup + args.steps):
+        idx = (np.arange(sample) + i * sample) % st.num_seqs
+        t = time.perf_counter()
+        oracle.decode(st.q[idx], kc, vc, st.block_tables[idx], st.context_lens[idx], wl.scale, wl.dtype)
+        dt = time.perf_counter() - t
+        if i >= args.warmup:
+            times.append(dt)
+            nbytes.append(int(st.context_lens[idx].sum()) * per_seq)
+    total_t = sum(times)
+    value = sum(nbytes) / total_t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_t / len(times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "sample": f"{sample} sequences per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{sample} of {st.num_seqs} sequences per step, rotating"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_457_b200 as pa
+
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    pa.load_library()
+
+    wl = make_workload(args.workload, rank)
+    if len(wl.steps) != 1:
+        steps_used = wl.steps[1:2]  # steady-state decode step of the multi-step workload
+    else:
+        steps_used = wl.steps
+    st = steps_used[0]
+    tdt = torch.float16 if wl.dtype == "fp16" else torch.bfloat16
+
+    def dev_bits(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(tdt)
+
+    k_cache = dev_bits(wl.k_cache)
+    v_cache = dev_bits(wl.v_cache)
+    if len(wl.steps) != 1:  # bring the cache to the state before the timed step
+        for prev in wl.steps[:1]:
+            pa.write_kv(dev_bits(prev.k_new), dev_bits(prev.v_new), k_cache, v_cache,
+                        torch.from_numpy(prev.slot_mapping).to(device))
+    q = dev_bits(st.q)
+    k_new = dev_bits(st.k_new)
+    v_new = dev_bits(st.v_new)
+    slots = torch.from_numpy(st.slot_mapping).to(device)
+    tables = torch.from_numpy(st.block_tables).to(device)
+    lens = torch.from_numpy(st.context_lens).to(device)
+    out = torch.empty_like(q)
+    mcl = st.max_context_len
+    part = args.partition_tokens
+    ws_bytes = pa.decode_workspace_size(st.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                        mcl, part)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+
+    def step(ev=None):
+        pa.write_kv(k_new, v_new, k_cache, v_cache, slots)
+        if ev is not None:
+            ev[0].record()
+        pa.decode(q, k_cache, v_cache, tables, lens, wl.scale, max_context_len=mcl, out=out,
+                  partition_tokens=part, workspace=ws)
+        if ev is not None:
+            ev[1].record()
+
+    kv_b, alg_b = step_bytes(wl, st)
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0, "device status after setup"
+
+    sampler = ClockSampler(device).start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = pa.launch_count()
+    wall0 = time.perf_counter()
+    t_start.record()
+    for i in range(args.steps):
+        step(dec_events[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    launches = pa.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_events)
+    status = pa.device_status()
+
+    # ---- end to end through the public API: pinned host inputs -> device -> step -> host output
+    e2e = None
+    if not args.no_e2e:
+        host = {n: torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else a)
+                .pin_memory() for n, a in (("q", st.q), ("k", st.k_new), ("v", st.v_new), ("slots", st.slot_mapping),
+                                           ("tables", st.block_tables), ("lens", st.context_lens))}
+        out_host = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+        dslots, dtables, dlens = torch.empty_like(slots), torch.empty_like(tables), torch.empty_like(lens)
+
+        def e2e_step():
+            dq.view(torch.int16).copy_(host["q"], non_blocking=True)
+            dk.view(torch.int16).copy_(host["k"], non_blocking=True)
+            dv.view(torch.int16).copy_(host["v"], non_blocking=True)
+            dslots.copy_(host["slots"], non_blocking=True)
+            dtables.copy_(host["tables"], non_blocking=True)
+            dlens.copy_(host["lens"], non_blocking=True)
+            pa.write_kv(dk, dv, k_cache, v_cache, dslots)
+            pa.decode(dq, k_cache, v_cache, dtables, dlens, wl.scale, max_context_len=mcl, out=out,
+                      partition_tokens=part, workspace=ws)
+            out_host.copy_(out.view(torch.int16), non_blocking=True)
+
+        for _ in range(max(3, args.warmup // 4)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(world * kv_b * args.steps / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e2e_ms / args.steps, 4)}
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, dec_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, dec_ms = float(t[0].item()), float(t[1].item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, nseq, secs = cpu_oracle_rate(wl, st, args.cpu_sample_seconds)
+        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"first {nseq} of {st.num_seqs} sequences of one step, {secs:.1f} s, single thread"}
+
+    if rank == 0:
+        ms_step = elapsed_ms / args.steps
+        value = world * kv_b / (ms_step / 1e3) / 1e9
+        peak, peak_kind = measured_peak()
+        achieved = alg_b / (dec_ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "storage_dtype": wl.dtype, "data": "synthetic",
+            "seq_steps_per_s": round(world * st.num_seqs / (ms_step / 1e3), 1),
+            "frac_of_hbm_peak": round(value / world / peak, 4),
+            "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
+            "config": {"workload": wl.name, "description": wl.description, "num_seqs": st.num_seqs,
+                       "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                       "block_size": wl.block_size, "max_context_len": mcl,
+                       "partition_tokens": part or pa.decode_partition_tokens(
+                           st.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, mcl),
+                       "kv_bytes_per_step": kv_b, "parallelism": f"dp{world} (independent batches per GPU)",
+                       "l2": f"no flush: {kv_b / 1e9:.2f} GB of K/V per step, larger than the 126 MB L2"},
+            "roofline": {"bound": "hbm", "kernel": "pa_decode (partition + reduce kernels)",
+                         "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "algorithmic_bytes": alg_b, "ms_per_launch": round(dec_ms, 5)},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": sampler.summary(wall0, wall1), "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,184 @@
+/*
+ * pa_b200.h -- C ABI of the B200 (sm_100a) paged decode attention library.
+ *
+ * The operations come from web pages describing vLLM / PagedAttention:
+ *  - "4. vLLM核心机制：PagedAttention、Continuous Batching、动态批处理",
+ *    section 4.2: the KV cache is cut into fixed-size pages (16 or 32 tokens);
+ *    a per-sequence page table maps logical page i to any physical page of
+ *    the pool; attention walks the pages through the table; prefix pages may
+ *    be named by several tables.  Section 4.3: each decode iteration produces
+ *    the new token and the updated KV cache.
+ *  - "vLLM：大型语言模型推理优化的革命性突破", section 2.1: the attention kernel
+ *    indexes the scattered blocks through the table, with no data movement
+ *    and no zero padding.
+ * Grouped-query heads (several query heads reading one KV head) are part of
+ * the problem statement this library serves, not of the pages.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or retains them.  The library allocates no device memory on
+ *    any call; its only device state is one status word per device (a
+ *    statically allocated __device__ variable).
+ *  - Storage elements are 2-byte floats: PA_FLOAT16 (IEEE binary16) or
+ *    PA_BFLOAT16.  Strides are in ELEMENTS.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and returns a PA_* status.  A negative status means the
+ *    arguments were rejected on the host and nothing was launched (or the
+ *    launch itself failed: PA_ERR_CUDA, text in pa_last_cuda_error()).
+ *  - Problems that only the device can see (a block id outside the pool, a
+ *    context length outside the table, a slot outside the pool, a bounded
+ *    wait that ran out) set bits in the device status word and never trap;
+ *    read them with pa_get_device_status().
+ *  - Cache layout: k_cache and v_cache are [num_blocks][num_kv_heads]
+ *    [block_size][head_dim], contiguous, so one (block, kv head) slab of
+ *    block_size * head_dim elements is contiguous in memory.
+ *  - Supported shapes: head_dim in {64, 128}; block_size in {16, 32};
+ *    num_q_heads a multiple of num_kv_heads (query head hq reads kv head
+ *    hq / (num_q_heads / num_kv_heads)).  All tensor base pointers must be
+ *    16-byte aligned and every token/sequence stride a multiple of 8 elements.
+ */
+#ifndef PA_B200_H
+#define PA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- host status codes ---- */
+#define PA_OK 0
+#define PA_ERR_NULL (-1)        /* a required pointer is NULL */
+#define PA_ERR_DTYPE (-2)       /* dtype is not PA_FLOAT16 / PA_BFLOAT16 */
+#define PA_ERR_SHAPE (-3)       /* a size is negative or inconsistent */
+#define PA_ERR_ALIGN (-4)       /* a pointer or stride breaks the 16-byte rule */
+#define PA_ERR_UNSUPPORTED (-5) /* head_dim or block_size outside the supported set */
+#define PA_ERR_HEADS (-6)       /* num_q_heads is not a multiple of num_kv_heads */
+#define PA_ERR_WORKSPACE (-7)   /* workspace missing, too small or misaligned */
+#define PA_ERR_PARTITION (-8)   /* partition_tokens not a multiple of block_size or too large */
+#define PA_ERR_CUDA (-9)        /* a CUDA runtime call failed; see pa_last_cuda_error() */
+
+/* ---- device status bits (pa_get_device_status) ---- */
+#define PA_DEV_ERR_BLOCK_ID 0x1u    /* a table entry a sequence needs is outside [0, num_blocks) */
+#define PA_DEV_ERR_CONTEXT 0x2u     /* context_len < 0 or > block_table_stride * block_size */
+#define PA_DEV_ERR_CONTEXT_HINT 0x4u /* context_len > the max_context_len the call was given */
+#define PA_DEV_ERR_SLOT 0x8u        /* a slot_mapping entry >= num_blocks * block_size */
+#define PA_DEV_ERR_TIMEOUT 0x10u    /* a bounded wait on a bulk copy ran out */
+
+typedef enum { PA_FLOAT16 = 1, PA_BFLOAT16 = 2 } pa_dtype;
+
+/*
+ * pa_write_kv -- store this step's new K and V rows into their cache slots
+ * ("4. vLLM核心机制" section 4.3, with the page layout of section 4.2).
+ *
+ * For every token t < num_tokens and kv head h:
+ *   slot = slot_mapping[t];  if slot < 0 the token is skipped (padding);
+ *   k_cache[slot / block_size][h][slot % block_size][:] = k[t][h][:]
+ *   v_cache[...same...]                                  = v[t][h][:]
+ * The copy is bit for bit.
+ *
+ *   k, v           [num_tokens][num_kv_heads][head_dim]; token stride
+ *                  k_token_stride / v_token_stride, heads contiguous.
+ *   k_cache,v_cache [num_blocks][num_kv_heads][block_size][head_dim].
+ *   slot_mapping   int64 [num_tokens].
+ * Slots must be distinct (two tokens writing one slot race).  A slot
+ * >= num_blocks * block_size is skipped and sets PA_DEV_ERR_SLOT.
+ * num_tokens == 0 launches nothing and returns PA_OK.
+ */
+int pa_write_kv(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                int64_t num_tokens, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                int64_t num_blocks, int64_t k_token_stride, int64_t v_token_stride, int32_t dtype,
+                void *stream);
+
+/*
+ * pa_decode_partition_tokens -- the partition length pa_decode uses when
+ * called with partition_tokens == 0, for this problem size on the current
+ * device.  Returns a positive multiple of block_size, or a PA_ERR_* code.
+ */
+int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t head_dim, int32_t block_size, int32_t max_context_len);
+
+/*
+ * pa_decode_workspace_size -- bytes of device workspace pa_decode needs for
+ * these sizes (0 when no sequence can span more than one partition).
+ * partition_tokens as for pa_decode (0 = automatic).  Returns 0 on bad input.
+ */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t block_size, int32_t max_context_len, int32_t partition_tokens);
+
+/*
+ * pa_decode -- single-token decode attention over the block-paged KV cache
+ * ("4. vLLM核心机制" section 4.2; "vLLM：大型语言模型推理优化的革命性突破" 2.1).
+ *
+ * For every sequence s and query head hq, with h = hq / (num_q_heads /
+ * num_kv_heads) and L = context_lens[s]:
+ *   token j < L lives in physical block block_tables[s][j / block_size],
+ *   row j % block_size;
+ *   z_j = scale * <q[s][hq][:], K_j>;  w = softmax(z);  out[s][hq][:] = sum_j w_j V_j.
+ * Arithmetic is fp32 (storage values widened exactly); the result is rounded
+ * to nearest-even into out's storage type (= dtype).  L == 0 gives zeros.
+ *
+ *   q               [num_seqs][num_q_heads][head_dim], sequence stride q_seq_stride.
+ *   k_cache,v_cache as for pa_write_kv.
+ *   block_tables    int32 [num_seqs][block_table_stride]; only entries
+ *                   j < ceil(L / block_size) of row s are read.
+ *   context_lens    int32 [num_seqs].
+ *   out             [num_seqs][num_q_heads][head_dim], sequence stride out_seq_stride.
+ *   max_context_len host-side upper bound of every context_len; it sizes the
+ *                   split over the token axis.  A sequence above it (or above
+ *                   the table's capacity) gets a zero output row and sets
+ *                   PA_DEV_ERR_CONTEXT_HINT (or PA_DEV_ERR_CONTEXT).
+ *   partition_tokens tokens per work unit along the context (0 = automatic;
+ *                   otherwise a multiple of block_size, at most 32 * block_size).
+ *                   A sequence longer than one partition is processed as
+ *                   several units whose partial softmax states are merged
+ *                   in a fixed order by a second kernel; results are
+ *                   deterministic run to run.
+ *   workspace       device scratch of at least pa_decode_workspace_size()
+ *                   bytes, 16-byte aligned (may be NULL when that size is 0).
+ *                   Contents need no initialisation and are overwritten.
+ *                   Calls that run concurrently must not share one workspace.
+ * A table entry outside [0, num_blocks) is never dereferenced: the affected
+ * (sequence, head) rows are zeroed and PA_DEV_ERR_BLOCK_ID is set.
+ * num_seqs == 0 launches nothing and returns PA_OK.
+ */
+int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+              const int32_t *context_lens, float scale, void *out, int32_t num_seqs, int32_t num_q_heads,
+              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int64_t num_blocks,
+              int32_t block_table_stride, int32_t max_context_len, int64_t q_seq_stride, int64_t out_seq_stride,
+              int32_t partition_tokens, int32_t dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * pa_get_device_status -- wait for `stream`, then copy the current device's
+ * status word (PA_DEV_ERR_* bits accumulated by earlier calls) to
+ * *status_out; clear it when `clear` is non-zero.  Synchronises `stream`.
+ */
+int pa_get_device_status(uint32_t *status_out, int32_t clear, void *stream);
+
+/* pa_status_string -- static text for a PA_* status code. */
+const char *pa_status_string(int32_t status);
+
+/* pa_last_cuda_error -- text of the last CUDA failure seen by this thread ("" if none). */
+const char *pa_last_cuda_error(void);
+
+/* pa_launch_count -- kernels this library has launched in this process (all devices). */
+uint64_t pa_launch_count(void);
+
+/*
+ * pa_debug_wait_timeout -- self-test of the bounded wait used by the decode
+ * kernel: launches one warp that waits on a shared-memory barrier that
+ * nothing will ever complete, giving up after limit_ns nanoseconds (clamped
+ * to [1e3, 1e9]); the kernel then sets PA_DEV_ERR_TIMEOUT and returns.
+ * Touches no caller memory.
+ */
+int pa_debug_wait_timeout(int64_t limit_ns, void *stream);
+
+/* pa_version -- library ABI version (major * 10000 + minor * 100 + patch). */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_B200_H */

@@ -1,0 +1,105 @@
+"""The C ABI library on a machine without a GPU: it builds, loads, exports every symbol the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_457_b200 as pa
+from paged_kv_cache_457_b200 import build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _has_gpu():
+    import torch
+    return torch.cuda.is_available()
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return pa.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("pa_write_kv", "pa_decode", "pa_decode_workspace_size", "pa_get_device_status"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+    assert set(names) == set(pa.EXPORTED_SYMBOLS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.pa_version() == 100
+    assert lib.pa_status_string(0) == b"ok"
+    for code in range(-9, 0):
+        assert lib.pa_status_string(code) != b"unknown status"
+
+
+def _decode(lib, **over):
+    args = dict(q=16, k=16, v=16, bt=16, cl=16, scale=0.1, out=16, S=2, hq=4, hkv=2, d=128, bs=16, nb=10, mb=4,
+                mcl=40, qs=512, os_=512, part=0, dtype=1, ws=None, wsb=0, stream=None)
+    args.update(over)
+    return lib.pa_decode(args["q"], args["k"], args["v"], args["bt"], args["cl"], args["scale"], args["out"],
+                         args["S"], args["hq"], args["hkv"], args["d"], args["bs"], args["nb"], args["mb"],
+                         args["mcl"], args["qs"], args["os_"], args["part"], args["dtype"], args["ws"], args["wsb"],
+                         args["stream"])
+
+
+def test_host_validation_of_decode(lib):
+    assert _decode(lib, d=96) == -5
+    assert _decode(lib, bs=8) == -5
+    assert _decode(lib, hq=6, hkv=4) == -6
+    assert _decode(lib, dtype=3) == -2
+    assert _decode(lib, S=-1) == -3
+    assert _decode(lib, mcl=-1) == -3
+    assert _decode(lib, qs=100) == -3
+    assert _decode(lib, q=None) == -1
+    assert _decode(lib, q=24) == -4  # misaligned pointer
+    assert _decode(lib, qs=516) == -4  # stride not a multiple of 8
+    if not _has_gpu():  # never launch on the fake pointers used here
+        assert _decode(lib) == -9  # valid arguments reach CUDA, absent here: reported, not thrown
+    assert _decode(lib, S=0) == 0  # empty batch: nothing to do, no CUDA call
+
+
+def test_host_validation_of_write(lib):
+    w = lib.pa_write_kv
+    # every call below fails validation (or has no tokens) before any CUDA call
+    assert w(16, 16, 16, 16, 16, 4, 2, 128, 16, 10, 256, 256, 5, None) == -2
+    assert w(16, 16, 16, 16, 16, 4, 2, 96, 16, 10, 256, 256, 1, None) == -5
+    assert w(16, 16, 16, 16, None, 4, 2, 128, 16, 10, 256, 256, 1, None) == -1
+    assert w(16, 16, 16, 16, 16, 4, 2, 128, 16, 10, 100, 256, 1, None) == -3
+    assert w(16, 16, 16, 20, 16, 4, 2, 128, 16, 10, 256, 256, 1, None) == -4
+    assert w(16, 16, 16, 16, 16, 0, 2, 128, 16, 10, 256, 256, 1, None) == 0
+
+
+def test_library_is_sm100a_only():
+    cmd = build_lib.command()
+    assert "arch=compute_100a,code=sm_100a" in cmd
+    assert not any("sm_90" in c or "compute_90" in c for c in cmd)
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(2, 4, 128, dtype=torch.float16)
+    with pytest.raises(pa.PagedAttentionError):
+        pa.decode(x, x, x, torch.zeros(2, 1, dtype=torch.int32), torch.zeros(2, dtype=torch.int32), 0.1,
+                  max_context_len=1)

@@ -1,0 +1,97 @@
+"""CUDA path against the fp64 oracle, element by element (needs a B200)."""
+import gc
+import json
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from gpu_util import DeviceState, compare, host_bits, oracle_step, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _free():
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+    yield
+    _free()
+
+
+@pytest.mark.parametrize("name", ["tiny_decode", "llama2_7b_decode", "gqa_llama3_decode", "long_context_splitk"])
+def test_full_config_write_and_decode(name):
+    """Full-size single-step workloads: the KV write is bit-exact over the whole pool and every
+    output element is within tolerance of the oracle, in the launch configuration the bench times."""
+    wl = W.NAMED[name]()
+    st = wl.steps[0]
+    dev = DeviceState(wl)
+    dev.write(st)
+    out = dev.decode(st)
+    torch.cuda.synchronize()
+    import paged_kv_cache_457_b200 as pa
+    assert pa.device_status() == 0
+    kc, vc, ref = oracle_step(wl, wl.k_cache, wl.v_cache, st)
+    assert np.array_equal(host_bits(dev.k_cache), kc), "k_cache differs from the oracle's scatter"
+    assert np.array_equal(host_bits(dev.v_cache), vc), "v_cache differs from the oracle's scatter"
+    stats = compare(out, ref, wl.dtype, what=name)
+    print(name, json.dumps(stats))
+    del dev, kc, vc
+    _free()
+
+
+def test_shared_prefix_steps():
+    """16 continuous-batching steps over shared-prefix groups (retire + join after step 8):
+    every step's cache is bit-exact; outputs are checked in full on steps 0, 8 and 15 and on
+    eight sampled sequences on the others."""
+    wl = W.shared_prefix()
+    dev = DeviceState(wl)
+    kc, vc = wl.k_cache, wl.v_cache
+    rng = np.random.default_rng(0)
+    for i, st in enumerate(wl.steps):
+        dev.write(st)
+        out = dev.decode(st)
+        seqs = None if i in (0, 8, 15) else np.sort(rng.choice(st.num_seqs, 8, replace=False))
+        kc, vc, ref = oracle_step(wl, kc, vc, st, seqs)
+        got = out if seqs is None else out[seqs]
+        compare(got, ref, wl.dtype, what=f"step {i}")
+        if i in (0, 8, 15):
+            assert np.array_equal(host_bits(dev.k_cache), kc), f"k_cache differs at step {i}"
+            assert np.array_equal(host_bits(dev.v_cache), vc), f"v_cache differs at step {i}"
+    import paged_kv_cache_457_b200 as pa
+    assert pa.device_status() == 0
+
+
+SMALL = [  # (hq, hkv, d, bs, dtype)
+    (4, 4, 64, 16, "fp16"),
+    (8, 8, 128, 16, "bf16"),
+    (8, 2, 128, 32, "fp16"),
+    (8, 1, 64, 32, "bf16"),
+    (6, 2, 128, 16, "bf16"),
+    (12, 4, 64, 16, "fp16"),
+    (16, 2, 128, 16, "bf16"),
+    (2, 2, 128, 32, "bf16"),
+]
+LENS = [1, 2, 15, 16, 17, 31, 33, 100, 257, 512, 513, 777, 1024, 1025]
+
+
+@pytest.mark.parametrize("hq,hkv,d,bs,dtype", SMALL)
+@pytest.mark.parametrize("partition", [0, 32, 64, 512])
+def test_small_shapes(hq, hkv, d, bs, dtype, partition):
+    """Every supported head dim / block size / group size / dtype, ragged lengths spanning
+    several tiles and partitions, explicit partition sizes (split-K) including one tile."""
+    if partition and partition % bs:
+        pytest.skip("partition must be a multiple of block_size")
+    wl = W.custom(seed=hq * 1000 + hkv * 100 + d + bs, num_seqs=len(LENS), num_q_heads=hq, num_kv_heads=hkv,
+                  head_dim=d, block_size=bs, lens=LENS, dtype=dtype)
+    st = wl.steps[0]
+    dev = DeviceState(wl)
+    dev.write(st)
+    out = dev.decode(st, partition_tokens=partition)
+    _, _, ref = oracle_step(wl, wl.k_cache, wl.v_cache, st)
+    compare(out, ref, dtype, what=f"{hq}/{hkv} d{d} bs{bs} {dtype} part {partition}")
