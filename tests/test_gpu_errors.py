@@ -67,7 +67,7 @@ def test_slot_out_of_range_is_skipped_and_flagged():
     bad = to_dev_index(np.array([wl.num_blocks * 16, -1], dtype=np.int64))
     pa.write_kv(k, k, dev.k_cache, dev.v_cache, bad)
     assert pa.device_status() == pa.DEV_ERR_SLOT
-    assert torch.equal(before, dev.k_cache)
+    assert torch.equal(before.view(torch.int16), dev.k_cache.view(torch.int16))  # bits: the pool holds NaN
 
 
 def test_bounded_wait_times_out_with_status():
