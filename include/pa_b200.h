@@ -17,8 +17,9 @@
  * Conventions shared by every entry point
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never frees or retains them.  The library allocates no device memory on
- *    any call; its only device state is one status word per device (a
- *    statically allocated __device__ variable).
+ *    any call; its device state is statically allocated __device__ data: one
+ *    status word per device, and the fixed scratch array behind
+ *    pa_decode_static_workspace.
  *  - Storage elements are 2-byte floats: PA_FLOAT16 (IEEE binary16) or
  *    PA_BFLOAT16.  Strides are in ELEMENTS.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
@@ -58,6 +59,10 @@ extern "C" {
 #define PA_ERR_WORKSPACE (-7)   /* workspace missing, too small or misaligned */
 #define PA_ERR_PARTITION (-8)   /* partition_tokens not a multiple of block_size or too large */
 #define PA_ERR_CUDA (-9)        /* a CUDA runtime call failed; see pa_last_cuda_error() */
+#define PA_ERR_STATIC_WORKSPACE (-10) /* the problem needs more scratch than PA_STATIC_WORKSPACE_BYTES */
+
+/* Size of the fixed scratch array behind pa_decode_static_workspace (32 MiB). */
+#define PA_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
 
 /* ---- device status bits (pa_get_device_status) ---- */
 #define PA_DEV_ERR_BLOCK_ID 0x1u    /* a table entry a sequence needs is outside [0, num_blocks) */
@@ -173,6 +178,44 @@ uint64_t pa_launch_count(void);
  * Touches no caller memory.
  */
 int pa_debug_wait_timeout(int64_t limit_ns, void *stream);
+
+/*
+ * pa_decode_static_workspace -- pa_decode for callers that cannot allocate
+ * device memory.  The pages have no counterpart to this entry point; it
+ * exists for the library's users.
+ *
+ * Some callers may not call cudaMalloc (or any allocator) at run time: a
+ * plugin inside a host framework that owns every device allocation, or a
+ * server that fixes its memory budget at start-up and must not allocate,
+ * fragment memory or pay an allocator's implicit device synchronisation in
+ * the middle of a step.  Such callers cannot provide pa_decode's workspace.
+ * This variant takes the same arguments as pa_decode minus the workspace
+ * and uses instead a scratch array of PA_STATIC_WORKSPACE_BYTES (32 MiB)
+ * compiled into the library as a static __device__ variable.  Every GPU on
+ * which the library is loaded holds that array until the process exits.
+ *
+ * - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - A problem whose split-context scratch (pa_decode_workspace_size for the
+ *   same sizes and partition_tokens) exceeds PA_STATIC_WORKSPACE_BYTES is
+ *   rejected with PA_ERR_STATIC_WORKSPACE before anything is launched; use
+ *   pa_decode with a caller workspace, or a larger partition_tokens.
+ * - The first call on each device looks up the array's device address with
+ *   cudaGetSymbolAddress while that device is current and caches it; make
+ *   that first call before any stream capture begins.
+ * - All calls on a device share the one array, and it keeps whatever the
+ *   last call left there.  The decode kernels write every scratch entry
+ *   before reading it, so nothing needs clearing between calls; but two
+ *   calls that can run at the same time on the GPU (different streams with
+ *   no ordering between them) race on the array and may corrupt each
+ *   other's results.  Order them on one stream, or use pa_decode.
+ * Results equal pa_decode's for the same arguments.
+ */
+int pa_decode_static_workspace(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_tables, const int32_t *context_lens, float scale, void *out,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t block_size, int64_t num_blocks, int32_t block_table_stride,
+                               int32_t max_context_len, int64_t q_seq_stride, int64_t out_seq_stride,
+                               int32_t partition_tokens, int32_t dtype, void *stream);
 
 /* pa_version -- library ABI version (major * 10000 + minor * 100 + patch). */
 int32_t pa_version(void);

@@ -45,7 +45,7 @@ _DTYPES = {torch.float16: 1, torch.bfloat16: 2}
 EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_decode_partition_tokens", "pa_decode_workspace_size", "pa_decode",
     "pa_get_device_status", "pa_status_string", "pa_last_cuda_error", "pa_launch_count",
-    "pa_debug_wait_timeout", "pa_version",
+    "pa_debug_wait_timeout", "pa_version", "pa_decode_static_workspace",
 )
 
 
@@ -88,6 +88,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_launch_count.argtypes = []
         lib.pa_debug_wait_timeout.restype = ctypes.c_int
         lib.pa_debug_wait_timeout.argtypes = [i64, vp]
+        lib.pa_decode_static_workspace.restype = ctypes.c_int
+        lib.pa_decode_static_workspace.argtypes = [vp, vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i64, i32,
+                                                   i32, i64, i64, i32, i32, vp]
         lib.pa_version.restype = i32
         lib.pa_version.argtypes = []
         if path is None:

@@ -164,6 +164,33 @@ int launch_decode_d(const pa::DecodeArgs &args, int G, int sms, cudaStream_t str
   return PA_OK;
 }
 
+// Fixed scratch behind pa_decode_static_workspace, for callers that cannot
+// allocate.  In host code this name is only a stand-in for the device
+// variable: the kernels are given the address cudaGetSymbolAddress returns.
+static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
+void *g_static_workspace_addr[kMaxDevices] = {};
+
+// Device address of g_static_workspace on the current device, looked up on
+// the first call for that device (with that device current) and cached.
+int static_workspace_address(void **addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record(e);
+  if (dev < 0 || dev >= kMaxDevices) {
+    t_last_cuda_error = "device ordinal beyond the library's table";
+    return PA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_workspace_addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return record(e);
+    g_static_workspace_addr[dev] = p;
+  }
+  *addr = g_static_workspace_addr[dev];
+  return PA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -326,6 +353,9 @@ const char *pa_status_string(int32_t status) {
     case PA_ERR_WORKSPACE: return "workspace missing, smaller than pa_decode_workspace_size() or misaligned";
     case PA_ERR_PARTITION: return "partition_tokens must be a multiple of block_size and of 16, at most 32 blocks";
     case PA_ERR_CUDA: return "a CUDA runtime call failed (see pa_last_cuda_error)";
+    case PA_ERR_STATIC_WORKSPACE:
+      return "the problem needs more split-context scratch than the library's fixed 32 MiB array; "
+             "use pa_decode with a caller workspace or a larger partition_tokens";
     default: return "unknown status";
   }
 }
@@ -341,6 +371,27 @@ int pa_debug_wait_timeout(int64_t limit_ns, void *stream) {
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return PA_OK;
+}
+
+int pa_decode_static_workspace(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_tables, const int32_t *context_lens, float scale, void *out,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t block_size, int64_t num_blocks, int32_t block_table_stride,
+                               int32_t max_context_len, int64_t q_seq_stride, int64_t out_seq_stride,
+                               int32_t partition_tokens, int32_t dtype, void *stream) {
+  int rc = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len);
+  if (rc != PA_OK) return rc;
+  if (num_seqs > 0) {  // an empty batch needs no scratch and launches nothing
+    const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                 max_context_len, partition_tokens);
+    if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_STATIC_WORKSPACE;
+  }
+  void *scratch = nullptr;
+  rc = static_workspace_address(&scratch);
+  if (rc != PA_OK) return rc;
+  return pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, num_seqs, num_q_heads, num_kv_heads,
+                   head_dim, block_size, num_blocks, block_table_stride, max_context_len, q_seq_stride,
+                   out_seq_stride, partition_tokens, dtype, scratch, PA_STATIC_WORKSPACE_BYTES, stream);
 }
 
 int32_t pa_version(void) { return 100; }
