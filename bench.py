@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
+    ap.add_argument("--num-seqs", type=int, default=None, help="override (llama2/gqa workloads; profiling)")
+    ap.add_argument("--num-blocks", type=int, default=None, help="override (llama2/gqa workloads; profiling)")
     return ap.parse_args()
 
 
@@ -55,8 +57,13 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", 0)))
 
 
-def make_workload(name: str, rank: int):
-    return W.NAMED[name](seed=SEEDS[name] + 1000 * rank)
+def make_workload(name: str, rank: int, num_seqs=None, num_blocks=None):
+    kw = {}
+    if num_seqs is not None:
+        kw["num_seqs"] = num_seqs
+    if num_blocks is not None:
+        kw["num_blocks"] = num_blocks
+    return W.NAMED[name](seed=SEEDS[name] + 1000 * rank, **kw)
 
 
 def step_bytes(wl, st):
@@ -215,7 +222,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
     pa.load_library()
 
-    wl = make_workload(args.workload, rank)
+    wl = make_workload(args.workload, rank, args.num_seqs, args.num_blocks)
     if len(wl.steps) != 1:
         steps_used = wl.steps[1:2]  # steady-state decode step of the multi-step workload
     else:

@@ -9,9 +9,13 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <mutex>
+
+#include <cudaTypedefs.h>
 
 #include "pa_b200.h"
 #include "pa_kernels.cuh"
+#include "pa_mma.cuh"
 
 namespace {
 
@@ -54,21 +58,54 @@ int current_sms(int *sms_out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Query heads handled together by one work unit: the largest of 4, 2, 1
-// dividing the group size (a unit reads its K/V tiles once for all of them).
-int heads_per_unit(int group) { return (group % 4 == 0) ? 4 : (group % 2 == 0) ? 2 : 1; }
+// Query heads handled together by one work unit (a unit reads its K/V tiles
+// once for all of them).  Groups of 1 or 2 run on the CUDA-core kernel; larger
+// groups run on the tensor-core kernel, whose units take up to 8 query heads
+// (the largest divisor of the group size not above 8).
+bool uses_mma(int group) { return group >= 3; }
+int heads_per_unit(int group) {
+  if (!uses_mma(group)) return group;
+  for (int c = 8; c > 1; --c)
+    if (group % c == 0) return c;
+  return 1;
+}
 
-// Per-head-dim launch shape of the partition kernel.
+// Per-head-dim launch shape of the partition kernel (warps per block, ring
+// depth per warp); overridable at build time for tuning sweeps.
+#ifndef PA_D128_WARPS
+#define PA_D128_WARPS 4
+#endif
+#ifndef PA_D128_STAGES
+#define PA_D128_STAGES 2
+#endif
+#ifndef PA_D64_WARPS
+#define PA_D64_WARPS 4
+#endif
+#ifndef PA_D64_STAGES
+#define PA_D64_STAGES 4
+#endif
 template <int D>
 struct Shape;
 template <>
 struct Shape<128> {
-  static constexpr int WARPS = 4, STAGES = 3;
+  static constexpr int WARPS = PA_D128_WARPS, STAGES = PA_D128_STAGES;
 };
 template <>
 struct Shape<64> {
-  static constexpr int WARPS = 4, STAGES = 4;
+  static constexpr int WARPS = PA_D64_WARPS, STAGES = PA_D64_STAGES;
 };
+
+#ifndef PA_MMA_WARPS
+#define PA_MMA_WARPS 4
+#endif
+#ifndef PA_MMA_STAGES
+#define PA_MMA_STAGES 2
+#endif
+constexpr int kMmaWarps = PA_MMA_WARPS, kMmaStages = PA_MMA_STAGES;
+template <int D>
+constexpr int mma_smem() {
+  return 1024 + kMmaWarps * kMmaStages * (2 * pa::TILE * D * 2 + 8);
+}
 
 template <int D>
 constexpr int partition_smem() {
@@ -76,10 +113,11 @@ constexpr int partition_smem() {
          Shape<D>::WARPS * Shape<D>::STAGES * 2 * pa::TILE * D * 2;
 }
 
-int warps_per_sm_estimate(int head_dim) {
+int warps_per_sm_estimate(int head_dim, bool mma) {
   // resident warps per SM that the shared-memory budget of the partition kernel allows
-  const int smem = head_dim == 128 ? partition_smem<128>() : partition_smem<64>();
-  const int warps = head_dim == 128 ? Shape<128>::WARPS : Shape<64>::WARPS;
+  const int smem = mma ? (head_dim == 128 ? mma_smem<128>() : mma_smem<64>())
+                       : (head_dim == 128 ? partition_smem<128>() : partition_smem<64>());
+  const int warps = mma ? kMmaWarps : (head_dim == 128 ? Shape<128>::WARPS : Shape<64>::WARPS);
   const int ctas = std::max(1, (227 * 1024) / (smem + 1024));
   return ctas * warps;
 }
@@ -91,21 +129,23 @@ int resolve_partition(int num_seqs, int num_q_heads, int num_kv_heads, int head_
       return PA_ERR_PARTITION;
     return requested;
   }
+  // Measured on B200: 16 blocks per unit suit the CUDA-core kernel, 8 the
+  // tensor-core kernel (its tiles go faster, so units must be more numerous).
   const int group = num_q_heads / num_kv_heads;
+  const bool mma = uses_mma(group);
   const long long base_units = (long long)num_seqs * num_kv_heads * (group / heads_per_unit(group));
-  const long long want = 2LL * sms * warps_per_sm_estimate(head_dim);
-  const int cap = 32 * block_size;
+  const long long want = (long long)sms * warps_per_sm_estimate(head_dim, mma);
   const int ctx = std::max(max_context_len, 1);
-  int part = cap;
-  // shrink until the (rough) number of units fills the GPU twice over; a
-  // context that fits one partition is never split
+  int part = (mma ? 8 : 16) * block_size;
+  // shrink while the (rough) number of units would not give every resident warp one
   while (part > 2 * pa::TILE && part > block_size) {
     const long long mean_parts = std::max(1LL, ((long long)ctx / 2 + part - 1) / part);
     if (base_units * mean_parts >= want) break;
     part /= 2;
   }
+  // a context that fits one partition is never split
   const int fit = ((ctx + block_size - 1) / block_size) * block_size;
-  if (fit <= cap && fit <= part) part = std::max(fit, pa::TILE);
+  if (fit <= part) part = std::max(fit, pa::TILE);
   if (part % block_size) part = ((part + block_size - 1) / block_size) * block_size;
   return part;
 }
@@ -146,13 +186,110 @@ int launch_partition(const pa::DecodeArgs &args, int sms, cudaStream_t stream) {
   return PA_OK;
 }
 
+// ---- TMA tensor maps of the caches, viewed as [num_blocks * num_kv_heads * block_size rows][head_dim],
+// boxes of 16 rows x 64 elements (128 bytes) with the 128-byte swizzle.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder(int *rc) {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (!fn) {
+    t_last_cuda_error = err != cudaSuccess ? cudaGetErrorString(err) : "cuTensorMapEncodeTiled not available";
+    *rc = PA_ERR_CUDA;
+  }
+  return fn;
+}
+
+struct MapKey {
+  int dev;
+  const void *base;
+  long long rows;
+  int head_dim, dtype;
+  bool operator==(const MapKey &o) const {
+    return dev == o.dev && base == o.base && rows == o.rows && head_dim == o.head_dim && dtype == o.dtype;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool used;
+};
+MapEntry g_maps[32];
+int g_map_next = 0;
+
+int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, CUtensorMap *out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record(e);
+  const MapKey key{dev, base, rows, head_dim, dtype};
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto &m : g_maps)
+    if (m.used && m.key == key) {
+      *out = m.map;
+      return PA_OK;
+    }
+  int rc = PA_OK;
+  auto encode = tensor_map_encoder(&rc);
+  if (!encode) return rc;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)pa::TILE};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUresult r = encode(&map, dtype == PA_BFLOAT16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                            2, const_cast<void *>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")";
+    return PA_ERR_CUDA;
+  }
+  g_maps[g_map_next] = MapEntry{key, map, true};
+  g_map_next = (g_map_next + 1) % 32;
+  *out = map;
+  return PA_OK;
+}
+
 template <class E, int D>
-int launch_decode_d(const pa::DecodeArgs &args, int G, int sms, cudaStream_t stream) {
+int launch_mma(const pa::DecodeArgs &args, int dtype, int sms, cudaStream_t stream) {
+  const long long rows = args.num_blocks * args.num_kv_heads * args.block_size;
+  if (rows > 0xffffffffLL) return PA_ERR_SHAPE;  // beyond what a tensor map (and the row index) can address
+  CUtensorMap mk, mv;
+  int rc = cache_tensor_map(args.k_cache, rows, D, dtype, &mk);
+  if (rc != PA_OK) return rc;
+  rc = cache_tensor_map(args.v_cache, rows, D, dtype, &mv);
+  if (rc != PA_OK) return rc;
+  constexpr int SMEM = mma_smem<D>();
+  auto kernel = pa::decode_partition_mma_kernel<E, D, kMmaWarps, kMmaStages>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return record(e);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kMmaWarps * 32, SMEM);
+  if (e != cudaSuccess) return record(e);
+  per_sm = std::max(per_sm, 1);
+  const long long need = (args.n_slots + kMmaWarps - 1) / kMmaWarps;
+  const int grid = (int)std::max(1LL, std::min<long long>((long long)sms * per_sm, need));
+  kernel<<<grid, kMmaWarps * 32, SMEM, stream>>>(mk, mv, args);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return record(e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+template <class E, int D>
+int launch_decode_d(const pa::DecodeArgs &args, int dtype, int sms, cudaStream_t stream) {
   int rc;
-  switch (G) {
-    case 4: rc = launch_partition<E, D, 4>(args, sms, stream); break;
-    case 2: rc = launch_partition<E, D, 2>(args, sms, stream); break;
-    default: rc = launch_partition<E, D, 1>(args, sms, stream); break;
+  if (uses_mma(args.group)) {
+    rc = launch_mma<E, D>(args, dtype, sms, stream);
+  } else if (args.heads_per_unit == 2) {
+    rc = launch_partition<E, D, 2>(args, sms, stream);
+  } else {
+    rc = launch_partition<E, D, 1>(args, sms, stream);
   }
   if (rc != PA_OK || args.n_part_max <= 1) return rc;
   const long long warps = (long long)args.num_seqs * args.num_q_heads;
@@ -315,13 +452,14 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   a.n_part_max = n_part_max;
   a.group = group;
   a.n_chunks = group / G;
+  a.heads_per_unit = G;
   a.n_slots = (long long)n_part_max * num_seqs * num_kv_heads * a.n_chunks;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == PA_BFLOAT16;
   if (head_dim == 128)
-    return bf16 ? launch_decode_d<pa::BF16, 128>(a, G, sms, st) : launch_decode_d<pa::F16, 128>(a, G, sms, st);
-  return bf16 ? launch_decode_d<pa::BF16, 64>(a, G, sms, st) : launch_decode_d<pa::F16, 64>(a, G, sms, st);
+    return bf16 ? launch_decode_d<pa::BF16, 128>(a, dtype, sms, st) : launch_decode_d<pa::F16, 128>(a, dtype, sms, st);
+  return bf16 ? launch_decode_d<pa::BF16, 64>(a, dtype, sms, st) : launch_decode_d<pa::F16, 64>(a, dtype, sms, st);
 }
 
 int pa_get_device_status(uint32_t *status_out, int32_t clear, void *stream) {

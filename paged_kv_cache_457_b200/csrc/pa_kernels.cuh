@@ -31,7 +31,13 @@ constexpr int TILE = 16;  // tokens per bulk-copied tile
 __device__ unsigned int g_status = 0;
 
 // ---------------------------------------------------------------- element types
+__device__ __forceinline__ float dot8_f16(const uint32_t (&q)[4], const uint4 k, float c);
+__device__ __forceinline__ float dot8_bf16(const uint32_t (&q)[4], const uint4 k, float c);
+
 struct F16 {
+  static __device__ __forceinline__ float dot8(const uint32_t (&q)[4], const uint4 k, float c) {
+    return dot8_f16(q, k, c);
+  }
   static __device__ __forceinline__ void widen8(const uint4 w, float (&f)[8]) {
     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -49,6 +55,9 @@ struct F16 {
 };
 
 struct BF16 {
+  static __device__ __forceinline__ float dot8(const uint32_t (&q)[4], const uint4 k, float c) {
+    return dot8_bf16(q, k, c);
+  }
   static __device__ __forceinline__ void widen8(const uint4 w, float (&f)[8]) {
     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -122,10 +131,106 @@ struct DecodeArgs {
   float scale_log2;  // scale * log2(e): logits are kept in base-2 units
   int num_seqs, num_q_heads, num_kv_heads, block_size, table_stride;
   int max_context_len, part_tokens, n_part_max, group, n_chunks;
+  int heads_per_unit;  // query heads sharing one kv head handled by one unit (group / n_chunks)
 };
 
 __device__ __forceinline__ bool context_ok(const DecodeArgs &a, int L) {
   return L >= 0 && (long long)L <= (long long)a.table_stride * a.block_size && L <= a.max_context_len;
+}
+
+// One work unit: partition p of sequence s, kv head h, query heads
+// hq0 .. hq0 + heads_per_unit - 1.
+struct Unit {
+  int s, h, p, hq0, L, tok_begin, tok_end, blk_begin, nblk;
+  bool work;  // context valid and non-empty: tiles to stream
+};
+
+// A warp's static, strided list of unit slots.  Slot order is partition
+// index outermost, then sequence, kv head, query-head chunk; slot p of a
+// sequence is empty when p * part_tokens >= L (slot p = 0 always exists: it
+// zeroes the rows of empty or invalid sequences).
+struct UnitList {
+  long long base, nwarps, per_part, per_seq;
+  int lane;
+
+  __device__ __forceinline__ UnitList(const DecodeArgs &a, int warps_per_block) {
+    lane = threadIdx.x & 31;
+    nwarps = (long long)gridDim.x * warps_per_block;
+    per_seq = (long long)a.num_kv_heads * a.n_chunks;
+    per_part = (long long)a.num_seqs * per_seq;
+    base = (long long)blockIdx.x * warps_per_block + (threadIdx.x >> 5);
+  }
+
+  // Next non-empty slot (32 candidates per step, one per lane); -1 when none is left.
+  __device__ __forceinline__ long long next(const DecodeArgs &a, int &L_out) {
+    while (base < a.n_slots) {
+      const long long c = base + (long long)lane * nwarps;
+      bool live = false;
+      int Lc = 0;
+      if (c < a.n_slots) {
+        const int p = (int)(c / per_part);
+        const int s = (int)((c - (long long)p * per_part) / per_seq);
+        Lc = __ldg(a.context_lens + s);
+        live = (p == 0) || (context_ok(a, Lc) && (long long)p * a.part_tokens < Lc);
+      }
+      const unsigned m = __ballot_sync(FULL, live);
+      if (m) {
+        const int idx = __ffs(m) - 1;
+        L_out = __shfl_sync(FULL, Lc, idx);
+        const long long slot = base + (long long)idx * nwarps;
+        base = slot + nwarps;
+        return slot;
+      }
+      base += 32LL * nwarps;
+    }
+    return -1;
+  }
+
+  __device__ __forceinline__ Unit describe(const DecodeArgs &a, long long slot, int L) const {
+    Unit u;
+    u.p = (int)(slot / per_part);
+    long long rem = slot - (long long)u.p * per_part;
+    u.s = (int)(rem / per_seq);
+    rem -= (long long)u.s * per_seq;
+    u.h = (int)(rem / a.n_chunks);
+    u.hq0 = u.h * a.group + (int)(rem - (long long)u.h * a.n_chunks) * a.heads_per_unit;
+    u.L = L;
+    u.work = context_ok(a, L) && L > 0;
+    u.tok_begin = u.p * a.part_tokens;
+    u.tok_end = u.work ? min(L, u.tok_begin + a.part_tokens) : u.tok_begin;
+    u.blk_begin = u.tok_begin / a.block_size;
+    u.nblk = (u.tok_end - u.tok_begin + a.block_size - 1) / a.block_size;  // <= 32
+    return u;
+  }
+};
+
+// The unit's table entry for this lane (block blk_begin + lane), or 0.
+__device__ __forceinline__ int unit_table_entry(const DecodeArgs &a, const Unit &u, int lane) {
+  return (u.work && lane < u.nblk) ? __ldg(a.block_tables + (long long)u.s * a.table_stride + u.blk_begin + lane) : 0;
+}
+
+// Status bits and zero rows for a unit that streams nothing (empty or invalid
+// context, or a table entry outside the pool).
+__device__ __forceinline__ void unit_without_tiles(const DecodeArgs &a, const Unit &u, bool bad_entry, int lane,
+                                                   int D) {
+  const int n_parts = u.work ? (u.L + a.part_tokens - 1) / a.part_tokens : 1;
+  if (lane == 0) {
+    if (!u.work && u.L != 0)
+      atomicOr(&g_status, (u.L < 0 || (long long)u.L > (long long)a.table_stride * a.block_size)
+                              ? PA_DEV_ERR_CONTEXT
+                              : PA_DEV_ERR_CONTEXT_HINT);
+    if (u.work && bad_entry) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
+  }
+  if (n_parts == 1) {
+    for (int i = lane; i < a.heads_per_unit * D / 8; i += 32) {
+      const int gg = i / (D / 8), c = i - gg * (D / 8);
+      *reinterpret_cast<uint4 *>(a.out + (long long)u.s * a.out_seq_stride + (long long)(u.hq0 + gg) * D + c * 8) =
+          make_uint4(0, 0, 0, 0);
+    }
+  } else if (lane < a.heads_per_unit) {
+    // a partial marked invalid: the merge kernel zeroes the row
+    a.ws_ml[((long long)u.s * a.num_q_heads + u.hq0 + lane) * a.n_part_max + u.p] = make_float2(-INFINITY, -1.f);
+  }
 }
 
 // Sums, over the lanes of one row group (lane bits 0..log2(2R)-1), R partial
@@ -148,15 +253,52 @@ __device__ __forceinline__ float row_group_reduce(float (&v)[R], int lane) {
   return v[0] + __shfl_xor_sync(FULL, v[0], 1);
 }
 
-// Each warp is an independent worker: it walks its own list of work units
-// (sequence s, kv head h, query-head chunk ch, partition p) and streams the
-// unit's 16-token K/V tiles through a private STAGES-deep ring of shared
-// memory buffers filled by bulk copies.  There is no block-level barrier.
+// Element-type specific arithmetic used by the partition kernel.
+//   dot8: sum of 8 products q_i * k_i of packed 2-byte values (4 words each),
+//         computed by the mixed-precision fma (2-byte inputs widened exactly,
+//         fp32 accumulation) so no separate conversion is issued.
+//   widen8: 8 packed values -> fp32.
+__device__ __forceinline__ float dot8_f16(const uint32_t (&q)[4], const uint4 k, float c) {
+  float d;
+  asm("{\n\t.reg .b16 q0, q1, k0, k1;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {q0, q1}, %1;\n\tmov.b32 {k0, k1}, %5;\n\tfma.rn.f32.f16 t, q0, k0, %9;\n\tfma.rn.f32.f16 t, q1, k1, t;\n\t"
+      "mov.b32 {q0, q1}, %2;\n\tmov.b32 {k0, k1}, %6;\n\tfma.rn.f32.f16 t, q0, k0, t;\n\tfma.rn.f32.f16 t, q1, k1, t;\n\t"
+      "mov.b32 {q0, q1}, %3;\n\tmov.b32 {k0, k1}, %7;\n\tfma.rn.f32.f16 t, q0, k0, t;\n\tfma.rn.f32.f16 t, q1, k1, t;\n\t"
+      "mov.b32 {q0, q1}, %4;\n\tmov.b32 {k0, k1}, %8;\n\tfma.rn.f32.f16 t, q0, k0, t;\n\tfma.rn.f32.f16 %0, q1, k1, t;\n\t}"
+      : "=f"(d)
+      : "r"(q[0]), "r"(q[1]), "r"(q[2]), "r"(q[3]), "r"(k.x), "r"(k.y), "r"(k.z), "r"(k.w), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float dot8_bf16(const uint32_t (&q)[4], const uint4 k, float c) {
+  float d;
+  asm("{\n\t.reg .b16 q0, q1, k0, k1;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {q0, q1}, %1;\n\tmov.b32 {k0, k1}, %5;\n\tfma.rn.f32.bf16 t, q0, k0, %9;\n\tfma.rn.f32.bf16 t, q1, k1, t;\n\t"
+      "mov.b32 {q0, q1}, %2;\n\tmov.b32 {k0, k1}, %6;\n\tfma.rn.f32.bf16 t, q0, k0, t;\n\tfma.rn.f32.bf16 t, q1, k1, t;\n\t"
+      "mov.b32 {q0, q1}, %3;\n\tmov.b32 {k0, k1}, %7;\n\tfma.rn.f32.bf16 t, q0, k0, t;\n\tfma.rn.f32.bf16 t, q1, k1, t;\n\t"
+      "mov.b32 {q0, q1}, %4;\n\tmov.b32 {k0, k1}, %8;\n\tfma.rn.f32.bf16 t, q0, k0, t;\n\tfma.rn.f32.bf16 %0, q1, k1, t;\n\t}"
+      : "=f"(d)
+      : "r"(q[0]), "r"(q[1]), "r"(q[2]), "r"(q[3]), "r"(k.x), "r"(k.y), "r"(k.z), "r"(k.w), "f"(c));
+  return d;
+}
+
+// Each warp is an independent worker: it walks its own static, strided list
+// of work units (UnitList) and streams each unit's 16-token K/V tiles through
+// a private STAGES-deep ring of shared-memory buffers filled by bulk copies.
+// There is no block-level barrier.  Used for groups of G <= 2 query heads per
+// kv head (CUDA cores).
 //
-// Within a tile, lane l reads 16 bytes (8 head dims) of rows
-// r*NGRP + l/LPR (r < R) of K and of V; q lives in registers as fp32 pre-
-// multiplied by scale*log2(e).  The online softmax keeps a running max m,
-// running sum and un-normalised output per query head.
+// Per tile, lane l copies 16 bytes (8 head dims) of rows r*NGRP + l/LPR
+// (r < R) of K and of V from the ring into registers, and the ring slot is
+// refilled at once, before any arithmetic, so the copies in flight never wait
+// on the math.  The next unit's table entries and query rows are loaded while
+// the current unit runs.  QK^T uses the mixed-precision fma (2-byte inputs,
+// fp32 accumulation); the 16 dot products are finished by a reduce-scatter
+// butterfly.  The online softmax keeps, per query head, a running maximum m
+// that is raised only when a logit exceeds it by more than RESCALE_SLACK
+// (base-2 units), so most tiles need no max reduction; m cancels between the
+// numerator and the denominator, and the weights stay below 2^RESCALE_SLACK.
+constexpr float RESCALE_SLACK = 8.f;
+
 template <class E, int D, int G, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32) decode_partition_kernel(const DecodeArgs a) {
   constexpr int LPR = D / 8;       // lanes covering one K/V row
@@ -181,93 +323,37 @@ __global__ void __launch_bounds__(WARPS * 32) decode_partition_kernel(const Deco
   const int grp = lane / LPR;
   const int cl = lane % LPR;
   const int my_tok = ((lane & (LPR - 2)) >> 1) * NGRP + grp;  // token whose logit this lane ends with
-
-  const long long nwarps = (long long)gridDim.x * WARPS;
-  const long long per_part = (long long)a.num_seqs * a.num_kv_heads * a.n_chunks;
-  const long long per_seq = (long long)a.num_kv_heads * a.n_chunks;
-  long long base = (long long)blockIdx.x * WARPS + warp;
   uint32_t iter = 0;  // tiles consumed by this warp so far: ring slot iter % STAGES, phase (iter / STAGES) & 1
 
+  UnitList list(a, WARPS);
+  auto fetch_q = [&](const Unit &u, uint4 (&qraw)[G]) {
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg)
+      qraw[gg] = u.work ? __ldg(reinterpret_cast<const uint4 *>(a.q + (long long)u.s * a.q_seq_stride +
+                                                                (long long)(u.hq0 + gg) * D + cl * 8))
+                        : make_uint4(0, 0, 0, 0);
+  };
+
+  int L0 = 0;
+  const long long first = list.next(a, L0);
+  if (first < 0) return;
+  Unit cur = list.describe(a, first, L0);
+  int ent = unit_table_entry(a, cur, lane);
+  uint4 qraw[G];
+  fetch_q(cur, qraw);
+
   while (true) {
-    // ---- next non-empty unit of this warp's static list, 32 candidates per step
-    long long slot = -1;
-    while (base < a.n_slots) {
-      const long long c = base + (long long)lane * nwarps;
-      bool live = false;
-      if (c < a.n_slots) {
-        const int p = (int)(c / per_part);
-        const int s = (int)((c - (long long)p * per_part) / per_seq);
-        const int L = __ldg(a.context_lens + s);
-        live = (p == 0) || (context_ok(a, L) && (long long)p * a.part_tokens < L);
-      }
-      const unsigned m = __ballot_sync(FULL, live);
-      if (m) {
-        slot = base + (long long)(__ffs(m) - 1) * nwarps;
-        base = slot + nwarps;
-        break;
-      }
-      base += 32LL * nwarps;
-    }
-    if (slot < 0) break;
-
-    const int p = (int)(slot / per_part);
-    long long rem = slot - (long long)p * per_part;
-    const int s = (int)(rem / per_seq);
-    rem -= (long long)s * per_seq;
-    const int h = (int)(rem / a.n_chunks);
-    const int ch = (int)(rem - (long long)h * a.n_chunks);
-    const int hq0 = h * a.group + ch * G;
-    const int L = __ldg(a.context_lens + s);
-    uint16_t *out_row = a.out + (long long)s * a.out_seq_stride + (long long)hq0 * D + cl * 8;
-
-    if (!context_ok(a, L) || L == 0) {  // only the p == 0 unit reaches here
-      if (lane == 0 && L != 0)
-        atomicOr(&g_status, (L < 0 || (long long)L > (long long)a.table_stride * a.block_size)
-                                ? PA_DEV_ERR_CONTEXT
-                                : PA_DEV_ERR_CONTEXT_HINT);
-      if (lane < LPR) {
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) *reinterpret_cast<uint4 *>(out_row + gg * D) = make_uint4(0, 0, 0, 0);
-      }
-      continue;
-    }
-
-    const int n_parts = (L + a.part_tokens - 1) / a.part_tokens;
-    const int tok_begin = p * a.part_tokens;
-    const int tok_end = min(L, tok_begin + a.part_tokens);
-    const int ntiles = (tok_end - tok_begin + TILE - 1) / TILE;
-    const int blk_begin = tok_begin / a.block_size;
-    const int nblk = (tok_end - tok_begin + a.block_size - 1) / a.block_size;  // <= 32
-
-    // ---- this unit's table entries, one per lane; validated before any copy
-    int ent = 0;
-    bool bad = false;
-    if (lane < nblk) {
-      ent = __ldg(a.block_tables + (long long)s * a.table_stride + blk_begin + lane);
-      bad = ent < 0 || (long long)ent >= a.num_blocks;
-    }
-    if (__any_sync(FULL, bad)) {
-      if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
-      if (n_parts == 1) {
-        if (lane < LPR) {
-#pragma unroll
-          for (int gg = 0; gg < G; ++gg) *reinterpret_cast<uint4 *>(out_row + gg * D) = make_uint4(0, 0, 0, 0);
-        }
-      } else if (lane == 0) {
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg)
-          a.ws_ml[((long long)s * a.num_q_heads + hq0 + gg) * a.n_part_max + p] = make_float2(-INFINITY, -1.f);
-      }
-      continue;
-    }
+    const int n_parts = cur.work ? (cur.L + a.part_tokens - 1) / a.part_tokens : 1;
+    const int ntiles = (cur.tok_end - cur.tok_begin + TILE - 1) / TILE;
+    const bool bad = __any_sync(FULL, cur.work && lane < cur.nblk && (ent < 0 || (long long)ent >= a.num_blocks));
 
     // ---- issue one tile: K and V rows [tok0, tok0 + 16) of (block, h) into ring slot it % STAGES
     auto issue = [&](int j, uint32_t it) {
-      const int tok0 = tok_begin + j * TILE;
-      const int phys = __shfl_sync(FULL, ent, tok0 / a.block_size - blk_begin);
+      const int tok0 = cur.tok_begin + j * TILE;
+      const int phys = __shfl_sync(FULL, ent, tok0 / a.block_size - cur.blk_begin);
       if (lane == 0) {
         const int st = (int)(it % STAGES);
-        const long long row0 = ((long long)phys * a.num_kv_heads + h) * a.block_size + (tok0 % a.block_size);
+        const long long row0 = ((long long)phys * a.num_kv_heads + cur.h) * a.block_size + (tok0 % a.block_size);
         unsigned char *dst = ring + st * STAGE_BYTES;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
@@ -275,144 +361,170 @@ __global__ void __launch_bounds__(WARPS * 32) decode_partition_kernel(const Deco
         bulk_copy_g2s(dst + TILE_BYTES, a.v_cache + row0 * D, TILE_BYTES, &bars[st]);
       }
     };
-    const int npro = ntiles < STAGES ? ntiles : STAGES;
+    const int npro = (cur.work && !bad) ? min(ntiles, STAGES) : 0;
     for (int j = 0; j < npro; ++j) issue(j, iter + j);
 
-    // ---- query rows (fp32, pre-scaled into base-2 logits)
-    float qf[G][8];
-#pragma unroll
-    for (int gg = 0; gg < G; ++gg) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.q + (long long)s * a.q_seq_stride +
-                                                            (long long)(hq0 + gg) * D + cl * 8));
-      E::widen8(w, qf[gg]);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) qf[gg][k] *= a.scale_log2;
+    // ---- look up and prefetch the next unit while those copies are in flight
+    int Ln = 0;
+    const long long nslot = list.next(a, Ln);
+    Unit nxt = cur;
+    int ent_n = 0;
+    uint4 qraw_n[G];
+    if (nslot >= 0) {
+      nxt = list.describe(a, nslot, Ln);
+      ent_n = unit_table_entry(a, nxt, lane);
+      fetch_q(nxt, qraw_n);
     }
 
-    float m[G], lsum[G], acc[G][8];
-#pragma unroll
-    for (int gg = 0; gg < G; ++gg) {
-      m[gg] = -INFINITY;
-      lsum[gg] = 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc[gg][k] = 0.f;
-    }
-
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = (int)(iter % STAGES);
-      const uint32_t parity = (iter / STAGES) & 1u;
-      const bool arrived = mbar_wait_bounded(&bars[st], parity, a.wait_limit_ns);
-      if (__any_sync(FULL, !arrived)) {
-        // A copy never landed: report, let every copy still in flight finish (bounded), stop.
-        if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
-        const int last = min(ntiles, j + STAGES);
-        for (int jj = j; jj < last; ++jj) {
-          const uint32_t it = iter + (jj - j);
-          mbar_wait_bounded(&bars[it % STAGES], (it / STAGES) & 1u, a.wait_limit_ns);
-        }
-        return;
-      }
-      const unsigned char *kt = ring + st * STAGE_BYTES;
-      const unsigned char *vt = kt + TILE_BYTES;
-      const int nvalid = min(TILE, tok_end - (tok_begin + j * TILE));
-
-      // QK^T: partial dots of this lane's 8 dims for its R rows, then the butterfly
-      float part[G][R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const uint4 kw = *reinterpret_cast<const uint4 *>(kt + ((r * NGRP + grp) * D + cl * 8) * 2);
-        float kf[8];
-        E::widen8(kw, kf);
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          float dot = qf[gg][0] * kf[0];
-#pragma unroll
-          for (int k = 1; k < 8; ++k) dot = fmaf(qf[gg][k], kf[k], dot);
-          part[gg][r] = dot;
-        }
-      }
-      const bool tok_live = my_tok < nvalid;
-      float pr[G][R];
-#pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        float z = row_group_reduce<R>(part[gg], lane);
-        z = tok_live ? z : -INFINITY;
-        float mt = z;
-        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
-        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 4));
-        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
-        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
-        if (mt > m[gg]) {  // warp-uniform: every lane holds the same mt and m
-          const float alpha = exp2f(m[gg] - mt);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) acc[gg][k] *= alpha;
-          lsum[gg] *= alpha;
-          m[gg] = mt;
-        }
-        const float pz = exp2f(z - m[gg]);
-        lsum[gg] += (lane & 1) ? 0.f : pz;
-#pragma unroll
-        for (int r = 0; r < R; ++r) pr[gg][r] = __shfl_sync(FULL, pz, grp * LPR + 2 * r);
-      }
-
-      // P.V: accumulate this lane's 8 dims over its R rows
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const uint4 vw = *reinterpret_cast<const uint4 *>(vt + ((r * NGRP + grp) * D + cl * 8) * 2);
-        float vf[8];
-        E::widen8(vw, vf);
-        if (nvalid < TILE) {  // rows past the sequence may hold anything (NaN): never let them in
-          const bool row_live = (r * NGRP + grp) < nvalid;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) vf[k] = row_live ? vf[k] : 0.f;
-        }
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) acc[gg][k] = fmaf(pr[gg][r], vf[k], acc[gg][k]);
-        }
-      }
-      __syncwarp();
-      if (j + STAGES < ntiles) issue(j + STAGES, iter + STAGES);
-      ++iter;
-    }
-
-    // ---- merge the row groups, total the running sums
-#pragma unroll
-    for (int gg = 0; gg < G; ++gg) {
-#pragma unroll
-      for (int off = LPR; off < 32; off <<= 1) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[gg][k] += __shfl_xor_sync(FULL, acc[gg][k], off);
-      }
-      float l = lsum[gg];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
-      lsum[gg] = l;
-    }
-
-    if (n_parts == 1) {
-      if (lane < LPR) {
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          float o[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) o[k] = acc[gg][k] / lsum[gg];
-          *reinterpret_cast<uint4 *>(out_row + gg * D) = narrow8<E>(o);
-        }
-      }
+    if (!cur.work || bad) {
+      unit_without_tiles(a, cur, bad, lane, D);
     } else {
+      uint16_t *out_row = a.out + (long long)cur.s * a.out_seq_stride + (long long)cur.hq0 * D + cl * 8;
+      uint32_t qw[G][4];
 #pragma unroll
       for (int gg = 0; gg < G; ++gg) {
-        const long long prow = ((long long)s * a.num_q_heads + hq0 + gg) * a.n_part_max + p;
-        if (lane < LPR) {
-          float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + prow * D + cl * 8);
-          dst[0] = make_float4(acc[gg][0], acc[gg][1], acc[gg][2], acc[gg][3]);
-          dst[1] = make_float4(acc[gg][4], acc[gg][5], acc[gg][6], acc[gg][7]);
+        qw[gg][0] = qraw[gg].x;
+        qw[gg][1] = qraw[gg].y;
+        qw[gg][2] = qraw[gg].z;
+        qw[gg][3] = qraw[gg].w;
+      }
+      float m[G], lsum[G];
+      float2 acc[G][4];
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        m[gg] = -INFINITY;
+        lsum[gg] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[gg][k] = make_float2(0.f, 0.f);
+      }
+
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = (int)(iter % STAGES);
+        const uint32_t parity = (iter / STAGES) & 1u;
+        const bool arrived = mbar_wait_bounded(&bars[st], parity, a.wait_limit_ns);
+        if (__any_sync(FULL, !arrived)) {
+          // A copy never landed: report, let every copy still in flight finish (bounded), stop.
+          if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
+          const int last = min(ntiles, j + STAGES);
+          for (int jj = j; jj < last; ++jj) {
+            const uint32_t it = iter + (jj - j);
+            mbar_wait_bounded(&bars[it % STAGES], (it / STAGES) & 1u, a.wait_limit_ns);
+          }
+          return;
         }
-        if (lane == 0) a.ws_ml[prow] = make_float2(m[gg], lsum[gg]);
+        // copy this lane's rows out of the ring, then hand the slot straight back to the copy engine
+        const unsigned char *kt = ring + st * STAGE_BYTES;
+        const unsigned char *vt = kt + TILE_BYTES;
+        uint4 kr[R], vr[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          kr[r] = *reinterpret_cast<const uint4 *>(kt + ((r * NGRP + grp) * D + cl * 8) * 2);
+          vr[r] = *reinterpret_cast<const uint4 *>(vt + ((r * NGRP + grp) * D + cl * 8) * 2);
+        }
+        __syncwarp();
+        if (j + STAGES < ntiles) issue(j + STAGES, iter + STAGES);
+        ++iter;
+        const int nvalid = min(TILE, cur.tok_end - (cur.tok_begin + j * TILE));
+        const bool tok_live = my_tok < nvalid;
+
+        // QK^T for this lane's R rows, the butterfly, scale, mask
+        float z[G];
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) {
+          float part[R];
+#pragma unroll
+          for (int r = 0; r < R; ++r) part[r] = E::dot8(qw[gg], kr[r], 0.f);
+          const float t = row_group_reduce<R>(part, lane) * a.scale_log2;
+          z[gg] = tok_live ? t : -INFINITY;
+        }
+        // softmax state: raise m only when some logit passes it by more than the slack
+        float pr[G][R];
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) {
+          if (__any_sync(FULL, z[gg] > m[gg] + RESCALE_SLACK)) {
+            float mt = z[gg];
+            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
+            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 4));
+            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
+            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
+            const float alpha = exp2f(m[gg] - mt);  // 0 on the first tile (m = -inf)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[gg][k] = make_float2(acc[gg][k].x * alpha, acc[gg][k].y * alpha);
+            lsum[gg] *= alpha;
+            m[gg] = mt;
+          }
+          const float pz = exp2f(z[gg] - m[gg]);
+          lsum[gg] += (lane & 1) ? 0.f : pz;
+#pragma unroll
+          for (int r = 0; r < R; ++r) pr[gg][r] = __shfl_sync(FULL, pz, grp * LPR + 2 * r);
+        }
+        // P.V over this lane's 8 dims and R rows (packed fp32 fma)
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float vf[8];
+          E::widen8(vr[r], vf);
+          if (nvalid < TILE) {  // rows past the sequence may hold anything (NaN): never let them in
+            const bool row_live = (r * NGRP + grp) < nvalid;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) vf[k] = row_live ? vf[k] : 0.f;
+          }
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) {
+            const float2 pp = make_float2(pr[gg][r], pr[gg][r]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[gg][k] = __ffma2_rn(pp, make_float2(vf[2 * k], vf[2 * k + 1]), acc[gg][k]);
+          }
+        }
+      }
+
+      // ---- merge the row groups, total the running sums, store
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+#pragma unroll
+        for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            acc[gg][k].x += __shfl_xor_sync(FULL, acc[gg][k].x, off);
+            acc[gg][k].y += __shfl_xor_sync(FULL, acc[gg][k].y, off);
+          }
+        }
+        float l = lsum[gg];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
+        lsum[gg] = l;
+      }
+      if (n_parts == 1) {
+        if (lane < LPR) {
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) {
+            float o[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              o[2 * k] = acc[gg][k].x / lsum[gg];
+              o[2 * k + 1] = acc[gg][k].y / lsum[gg];
+            }
+            *reinterpret_cast<uint4 *>(out_row + gg * D) = narrow8<E>(o);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) {
+          const long long prow = ((long long)cur.s * a.num_q_heads + cur.hq0 + gg) * a.n_part_max + cur.p;
+          if (lane < LPR) {
+            float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + prow * D + cl * 8);
+            dst[0] = make_float4(acc[gg][0].x, acc[gg][0].y, acc[gg][1].x, acc[gg][1].y);
+            dst[1] = make_float4(acc[gg][2].x, acc[gg][2].y, acc[gg][3].x, acc[gg][3].y);
+          }
+          if (lane == 0) a.ws_ml[prow] = make_float2(m[gg], lsum[gg]);
+        }
       }
     }
+
+    if (nslot < 0) break;
+    cur = nxt;
+    ent = ent_n;
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) qraw[gg] = qraw_n[gg];
   }
 }
 

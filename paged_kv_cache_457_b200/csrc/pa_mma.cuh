@@ -1,0 +1,304 @@
+// Tensor-core partition kernel for grouped-query decode: 3 to 8 query heads
+// of one unit share each K/V tile, so the query-group x tile product is a
+// real dense contraction and runs on mma.sync (m16n8k16, fp32 accumulation).
+//
+// Per 16-token tile, with the unit's query heads as the N = 8 columns:
+//   S^T[16 tokens x 8 heads]  = K[16 x d] . Q^T[d x 8]          (d/16 mma)
+//   O^T[d x 8 heads]         += V^T[d x 16 tokens] . P^T[16 x 8] (2 * d/16 mma)
+// K and V tiles arrive by 2-D TMA tensor copies with the 128-byte swizzle, so
+// the ldmatrix loads of both operands are free of bank conflicts.  P is
+// split into a 2-byte head and a 2-byte residual (P ~= Ph + Pl, relative
+// error ~2^-16) so the product keeps fp32-level accuracy although the mma
+// takes 2-byte operands; movmatrix turns P^T's accumulator layout into the
+// B operand layout.  The online softmax runs along the token (M) axis, per
+// head column, with the same lazy rescaling as the CUDA-core kernel.
+#pragma once
+
+#include <cuda.h>
+
+#include "pa_kernels.cuh"
+
+namespace pa {
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+template <class E>
+struct MmaOps;
+
+template <>
+struct MmaOps<F16> {
+  static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    mma_16816_f16(d, a, b0, b1);
+  }
+  // p0, p1 -> packed head (nearest) and packed residual
+  static __device__ __forceinline__ void split(float p0, float p1, uint32_t &hi, uint32_t &lo) {
+    __half2 h = __floats2half2_rn(p0, p1);
+    const float2 f = __half22float2(h);
+    __half2 l = __floats2half2_rn(p0 - f.x, p1 - f.y);
+    hi = *reinterpret_cast<uint32_t *>(&h);
+    lo = *reinterpret_cast<uint32_t *>(&l);
+  }
+};
+
+template <>
+struct MmaOps<BF16> {
+  static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    mma_16816_bf16(d, a, b0, b1);
+  }
+  // head = upper 16 bits (truncation; the residual is then exact in fp32)
+  static __device__ __forceinline__ void split(float p0, float p1, uint32_t &hi, uint32_t &lo) {
+    const uint32_t u0 = __float_as_uint(p0) & 0xffff0000u;
+    const uint32_t u1 = __float_as_uint(p1) & 0xffff0000u;
+    hi = (u0 >> 16) | u1;
+    __nv_bfloat162 l = __floats2bfloat162_rn(p0 - __uint_as_float(u0), p1 - __uint_as_float(u1));
+    lo = *reinterpret_cast<uint32_t *>(&l);
+  }
+};
+
+// Offset of 16-byte chunk c (8 head dims) of token row r in a tile stored as
+// D/64 boxes of [16 rows x 128 bytes] with the TMA 128-byte swizzle.
+__device__ __forceinline__ uint32_t swizzled(int r, int c) {
+  return (uint32_t)((c >> 3) * 2048 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <class E, int D, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32)
+    decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                                const DecodeArgs a) {
+  constexpr int KSTEPS = D / 16;  // 16-dim steps of QK^T, and 16-dim row tiles of O^T
+  constexpr int BOXES = D / 64;
+  constexpr uint32_t TILE_BYTES = TILE * D * 2;
+  constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;
+
+  extern __shared__ unsigned char smem_raw[];
+  // ring slots start on a 1024-byte boundary (the swizzle pattern repeats every 1024 bytes)
+  unsigned char *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  unsigned char *ring = smem + warp * STAGES * STAGE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + WARPS * STAGES * STAGE_BYTES) + warp * STAGES;
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
+    fence_mbar_init();
+    prefetch_tensor_map(&tmap_k);
+    prefetch_tensor_map(&tmap_v);
+  }
+  __syncwarp();
+
+  const int gid = lane >> 2;  // mma row group
+  const int tig = lane & 3;   // thread in group
+  // ldmatrix row addresses: lane supplies row (lane & 7) of matrix (lane >> 3)
+  const int mi = lane >> 3, mr = lane & 7;
+  const int ka_tok = 8 * (mi & 1) + mr, ka_c = mi >> 1;  // K as A (non-transposed)
+  const int va_tok = 8 * (mi >> 1) + mr, va_c = mi & 1;  // V^T as A (transposed)
+  const int G = a.heads_per_unit;
+  uint32_t iter = 0;
+
+  UnitList list(a, WARPS);
+  int L0 = 0;
+  const long long first = list.next(a, L0);
+  if (first < 0) return;
+  Unit cur = list.describe(a, first, L0);
+  int ent = unit_table_entry(a, cur, lane);
+
+  while (true) {
+    const int n_parts = cur.work ? (cur.L + a.part_tokens - 1) / a.part_tokens : 1;
+    const int ntiles = (cur.tok_end - cur.tok_begin + TILE - 1) / TILE;
+    const bool bad = __any_sync(FULL, cur.work && lane < cur.nblk && (ent < 0 || (long long)ent >= a.num_blocks));
+
+    auto issue = [&](int j, uint32_t it) {
+      const int tok0 = cur.tok_begin + j * TILE;
+      const int phys = __shfl_sync(FULL, ent, tok0 / a.block_size - cur.blk_begin);
+      if (lane == 0) {
+        const int st = (int)(it % STAGES);
+        const int row0 = (int)(((long long)phys * a.num_kv_heads + cur.h) * a.block_size + (tok0 % a.block_size));
+        unsigned char *dst = ring + st * STAGE_BYTES;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
+#pragma unroll
+        for (int b = 0; b < BOXES; ++b) {
+          tma_load_2d(dst + b * 2048, &tmap_k, b * 64, row0, &bars[st]);
+          tma_load_2d(dst + TILE_BYTES + b * 2048, &tmap_v, b * 64, row0, &bars[st]);
+        }
+      }
+    };
+    const bool streams = cur.work && !bad;
+    const int npro = streams ? min(ntiles, STAGES) : 0;
+    for (int j = 0; j < npro; ++j) issue(j, iter + j);
+
+    // Q^T as the B operand: b0 = Q[head gid][16ks + 2tig, +1], b1 = the same 8 dims later
+    uint32_t qb[KSTEPS][2];
+    {
+      const bool row_live = streams && gid < G;
+      const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q + (long long)cur.s * a.q_seq_stride +
+                                                                (long long)(cur.hq0 + (row_live ? gid : 0)) * D);
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        qb[ks][0] = row_live ? __ldg(qrow + 8 * ks + tig) : 0u;
+        qb[ks][1] = row_live ? __ldg(qrow + 8 * ks + 4 + tig) : 0u;
+      }
+    }
+
+    // look up the next unit and its table entries while the copies are in flight
+    int Ln = 0;
+    const long long nslot = list.next(a, Ln);
+    Unit nxt = cur;
+    int ent_n = 0;
+    if (nslot >= 0) {
+      nxt = list.describe(a, nslot, Ln);
+      ent_n = unit_table_entry(a, nxt, lane);
+    }
+
+    if (!streams) {
+      unit_without_tiles(a, cur, bad, lane, D);
+    } else {
+      // per lane: head columns ha = 2*tig and hb = 2*tig + 1
+      float o[KSTEPS][4];
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+      float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = (int)(iter % STAGES);
+        const uint32_t parity = (iter / STAGES) & 1u;
+        const bool arrived = mbar_wait_bounded(&bars[st], parity, a.wait_limit_ns);
+        if (__any_sync(FULL, !arrived)) {
+          if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
+          const int last = min(ntiles, j + STAGES);
+          for (int jj = j; jj < last; ++jj) {
+            const uint32_t it = iter + (jj - j);
+            mbar_wait_bounded(&bars[it % STAGES], (it / STAGES) & 1u, a.wait_limit_ns);
+          }
+          return;
+        }
+        const uint32_t kt = smem_addr(ring + st * STAGE_BYTES);
+        const uint32_t vt = kt + TILE_BYTES;
+        uint32_t kf[KSTEPS][4], vf[KSTEPS][4];
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          ldsm_x4(kf[ks], kt + swizzled(ka_tok, 2 * ks + ka_c));
+          ldsm_x4_trans(vf[ks], vt + swizzled(va_tok, 2 * ks + va_c));
+        }
+        __syncwarp();
+        if (j + STAGES < ntiles) issue(j + STAGES, iter + STAGES);
+        ++iter;
+        const int nvalid = min(TILE, cur.tok_end - (cur.tok_begin + j * TILE));
+
+        // S^T = K Q^T: s0 = (token gid, head ha), s1 = (gid, hb), s2 = (gid + 8, ha), s3 = (gid + 8, hb)
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) MmaOps<E>::mma(s, kf[ks], qb[ks][0], qb[ks][1]);
+        const bool lo_live = gid < nvalid, hi_live = gid + 8 < nvalid;
+        const float z0 = lo_live ? s[0] * a.scale_log2 : -INFINITY;
+        const float z1 = lo_live ? s[1] * a.scale_log2 : -INFINITY;
+        const float z2 = hi_live ? s[2] * a.scale_log2 : -INFINITY;
+        const float z3 = hi_live ? s[3] * a.scale_log2 : -INFINITY;
+
+        const bool need = z0 > ma + RESCALE_SLACK || z2 > ma + RESCALE_SLACK || z1 > mb + RESCALE_SLACK ||
+                          z3 > mb + RESCALE_SLACK;
+        if (__any_sync(FULL, need)) {
+          float ca = fmaxf(z0, z2), cb = fmaxf(z1, z3);
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            ca = fmaxf(ca, __shfl_xor_sync(FULL, ca, off));
+            cb = fmaxf(cb, __shfl_xor_sync(FULL, cb, off));
+          }
+          const float na = fmaxf(ma, ca), nb = fmaxf(mb, cb);
+          const float alpha_a = exp2f(ma - na), alpha_b = exp2f(mb - nb);  // 0 on the first tile
+#pragma unroll
+          for (int mt = 0; mt < KSTEPS; ++mt) {
+            o[mt][0] *= alpha_a;
+            o[mt][1] *= alpha_b;
+            o[mt][2] *= alpha_a;
+            o[mt][3] *= alpha_b;
+          }
+          la *= alpha_a;
+          lb *= alpha_b;
+          ma = na;
+          mb = nb;
+        }
+        const float p0 = exp2f(z0 - ma), p1 = exp2f(z1 - mb), p2 = exp2f(z2 - ma), p3 = exp2f(z3 - mb);
+        la += p0 + p2;
+        lb += p1 + p3;
+
+        // P^T (tokens x heads) in accumulator layout -> P as the B operand (k = tokens, n = heads)
+        uint32_t h01, l01, h23, l23;
+        MmaOps<E>::split(p0, p1, h01, l01);
+        MmaOps<E>::split(p2, p3, h23, l23);
+        const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+        const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+
+        if (nvalid < TILE) {  // V rows past the sequence may hold NaN: zero them (0 * NaN would leak in)
+          const uint32_t m_lo = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
+          const uint32_t m_hi =
+              (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
+#pragma unroll
+          for (int ks = 0; ks < KSTEPS; ++ks) {
+            vf[ks][0] &= m_lo;
+            vf[ks][1] &= m_lo;
+            vf[ks][2] &= m_hi;
+            vf[ks][3] &= m_hi;
+          }
+        }
+        // O^T += V^T P^T, head part then residual part
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          MmaOps<E>::mma(o[mt], vf[mt], bh0, bh1);
+          MmaOps<E>::mma(o[mt], vf[mt], bl0, bl1);
+        }
+      }
+
+      // ---- totals per head column (lanes with the same tig), then store
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        la += __shfl_xor_sync(FULL, la, off);
+        lb += __shfl_xor_sync(FULL, lb, off);
+      }
+      const int ha = 2 * tig, hb = 2 * tig + 1;
+      if (n_parts == 1) {
+        // normalise, narrow, transpose 8x8 blocks back to [head][dims]: lane then holds head gid, dims 2tig, 2tig+1
+        const float ia = 1.f / la, ib = 1.f / lb;
+        uint16_t *orow = a.out + (long long)cur.s * a.out_seq_stride + (long long)(cur.hq0 + gid) * D + 2 * tig;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          const uint32_t t0 = movmatrix_trans(E::narrow2(o[mt][0] * ia, o[mt][1] * ib));
+          const uint32_t t1 = movmatrix_trans(E::narrow2(o[mt][2] * ia, o[mt][3] * ib));
+          if (gid < G) {
+            *reinterpret_cast<uint32_t *>(orow + 16 * mt) = t0;
+            *reinterpret_cast<uint32_t *>(orow + 16 * mt + 8) = t1;
+          }
+        }
+      } else {
+        const long long row_a = ((long long)cur.s * a.num_q_heads + cur.hq0 + ha) * a.n_part_max + cur.p;
+        const long long row_b = row_a + a.n_part_max;
+#pragma unroll
+        for (int mt = 0; mt < KSTEPS; ++mt) {
+          const int d0 = 16 * mt + gid;
+          if (ha < G) {
+            a.ws_acc[row_a * D + d0] = o[mt][0];
+            a.ws_acc[row_a * D + d0 + 8] = o[mt][2];
+          }
+          if (hb < G) {
+            a.ws_acc[row_b * D + d0] = o[mt][1];
+            a.ws_acc[row_b * D + d0 + 8] = o[mt][3];
+          }
+        }
+        if (gid == 0) {
+          if (ha < G) a.ws_ml[row_a] = make_float2(ma, la);
+          if (hb < G) a.ws_ml[row_b] = make_float2(mb, lb);
+        }
+      }
+    }
+
+    if (nslot < 0) break;
+    cur = nxt;
+    ent = ent_n;
+  }
+}
+
+}  // namespace pa
