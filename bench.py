@@ -362,8 +362,7 @@ def main():
             "config": {"workload": wl.name, "description": wl.description, "num_seqs": st.num_seqs,
                        "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                        "block_size": wl.block_size, "max_context_len": mcl,
-                       "partition_tokens": part or pa.decode_partition_tokens(
-                           st.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size, mcl),
+                       "split": f"chunks of {part} tokens" if part else "balanced (one chunk of tiles per warp)",
                        "kv_bytes_per_step": kv_b, "parallelism": f"dp{world} (independent batches per GPU)",
                        "l2": f"no flush: {kv_b / 1e9:.2f} GB of K/V per step, larger than the 126 MB L2"},
             "roofline": {"bound": "hbm", "kernel": "pa_decode (partition + reduce kernels)",

@@ -57,7 +57,7 @@ extern "C" {
 #define PA_ERR_UNSUPPORTED (-5) /* head_dim or block_size outside the supported set */
 #define PA_ERR_HEADS (-6)       /* num_q_heads is not a multiple of num_kv_heads */
 #define PA_ERR_WORKSPACE (-7)   /* workspace missing, too small or misaligned */
-#define PA_ERR_PARTITION (-8)   /* partition_tokens not a multiple of block_size or too large */
+#define PA_ERR_PARTITION (-8)   /* partition_tokens negative or not a multiple of 16 */
 #define PA_ERR_CUDA (-9)        /* a CUDA runtime call failed; see pa_last_cuda_error() */
 #define PA_ERR_STATIC_WORKSPACE (-10) /* the problem needs more scratch than PA_STATIC_WORKSPACE_BYTES */
 
@@ -97,17 +97,9 @@ int pa_write_kv(const void *k, const void *v, void *k_cache, void *v_cache, cons
                 void *stream);
 
 /*
- * pa_decode_partition_tokens -- the partition length pa_decode uses when
- * called with partition_tokens == 0, for this problem size on the current
- * device.  Returns a positive multiple of block_size, or a PA_ERR_* code.
- */
-int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
-                                   int32_t head_dim, int32_t block_size, int32_t max_context_len);
-
-/*
  * pa_decode_workspace_size -- bytes of device workspace pa_decode needs for
- * these sizes (0 when no sequence can span more than one partition).
- * partition_tokens as for pa_decode (0 = automatic).  Returns 0 on bad input.
+ * these sizes and this partition_tokens (see pa_decode) on the current
+ * device.  It does not depend on the storage type.  Returns 0 on bad input.
  */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                 int32_t block_size, int32_t max_context_len, int32_t partition_tokens);
@@ -134,16 +126,23 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t n
  *                   split over the token axis.  A sequence above it (or above
  *                   the table's capacity) gets a zero output row and sets
  *                   PA_DEV_ERR_CONTEXT_HINT (or PA_DEV_ERR_CONTEXT).
- *   partition_tokens tokens per work unit along the context (0 = automatic;
- *                   otherwise a multiple of block_size, at most 32 * block_size).
- *                   A sequence longer than one partition is processed as
- *                   several units whose partial softmax states are merged
- *                   in a fixed order by a second kernel; results are
- *                   deterministic run to run.
+ *   partition_tokens how the work is cut.  The tiles of 16 tokens of every
+ *                   (sequence, kv head, group of up to 8 query heads) are laid
+ *                   in one stream, ordered by sequence, then head group, then
+ *                   position, and the stream is cut into chunks of
+ *                   consecutive tiles that the GPU's warps take in turn.
+ *                   0 = balanced: one chunk per resident warp, so every warp
+ *                   gets the same number of tiles whatever the length mix;
+ *                   otherwise a positive multiple of 16: chunks of
+ *                   partition_tokens / 16 tiles.  A sequence cut across chunks
+ *                   is finished by a second kernel that merges the partial
+ *                   softmax states in a fixed order: results are deterministic
+ *                   run to run for the same arguments and device.
  *   workspace       device scratch of at least pa_decode_workspace_size()
- *                   bytes, 16-byte aligned (may be NULL when that size is 0).
- *                   Contents need no initialisation and are overwritten.
- *                   Calls that run concurrently must not share one workspace.
+ *                   bytes, 16-byte aligned.  Contents need no initialisation
+ *                   and are overwritten.  Calls that run concurrently must not
+ *                   share one workspace.
+ * num_seqs is at most 32768.
  * A table entry outside [0, num_blocks) is never dereferenced: the affected
  * (sequence, head) rows are zeroed and PA_DEV_ERR_BLOCK_ID is set.
  * num_seqs == 0 launches nothing and returns PA_OK.

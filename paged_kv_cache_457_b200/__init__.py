@@ -24,7 +24,7 @@ import threading
 import torch
 
 __all__ = [
-    "PagedAttentionError", "write_kv", "decode", "decode_workspace_size", "decode_partition_tokens",
+    "PagedAttentionError", "write_kv", "decode", "decode_workspace_size",
     "device_status", "launch_count", "debug_wait_timeout", "library_path", "load_library", "EXPORTED_SYMBOLS",
     "DEV_ERR_BLOCK_ID", "DEV_ERR_CONTEXT", "DEV_ERR_CONTEXT_HINT", "DEV_ERR_SLOT", "DEV_ERR_TIMEOUT",
 ]
@@ -43,7 +43,7 @@ DEV_ERR_TIMEOUT = 0x10
 _DTYPES = {torch.float16: 1, torch.bfloat16: 2}
 
 EXPORTED_SYMBOLS = (
-    "pa_write_kv", "pa_decode_partition_tokens", "pa_decode_workspace_size", "pa_decode",
+    "pa_write_kv", "pa_decode_workspace_size", "pa_decode",
     "pa_get_device_status", "pa_status_string", "pa_last_cuda_error", "pa_launch_count",
     "pa_debug_wait_timeout", "pa_version", "pa_decode_static_workspace",
 )
@@ -71,8 +71,6 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
         lib.pa_write_kv.restype = ctypes.c_int
         lib.pa_write_kv.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, i64, i64, i32, vp]
-        lib.pa_decode_partition_tokens.restype = i32
-        lib.pa_decode_partition_tokens.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.pa_decode_workspace_size.restype = sz
         lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32]
         lib.pa_decode.restype = ctypes.c_int
@@ -151,13 +149,6 @@ def write_kv(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: t
 
 
 _workspaces: dict = {}
-
-
-def decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len) -> int:
-    rc = load_library().pa_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                                   max_context_len)
-    _check(rc if rc < 0 else 0, "pa_decode_partition_tokens")
-    return int(rc)
 
 
 def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,

@@ -58,9 +58,9 @@ int current_sms(int *sms_out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Query heads handled together by one work unit (a unit reads its K/V tiles
-// once for all of them).  Groups of 1 or 2 run on the CUDA-core kernel; larger
-// groups run on the tensor-core kernel, whose units take up to 8 query heads
+// Query heads handled together by one head chunk (the K/V tiles are read once
+// for all of them).  Groups of 1 or 2 run on the CUDA-core kernel; larger
+// groups run on the tensor-core kernel, whose chunks take up to 8 query heads
 // (the largest divisor of the group size not above 8).
 bool uses_mma(int group) { return group >= 3; }
 int heads_per_unit(int group) {
@@ -70,119 +70,123 @@ int heads_per_unit(int group) {
   return 1;
 }
 
-// Per-head-dim launch shape of the partition kernel (warps per block, ring
-// depth per warp); overridable at build time for tuning sweeps.
-#ifndef PA_D128_WARPS
-#define PA_D128_WARPS 4
+// Launch shape of the split kernels (warps per block, ring slots per warp);
+// overridable at build time for tuning sweeps.
+#ifndef PA_WARPS
+#define PA_WARPS 4
 #endif
-#ifndef PA_D128_STAGES
-#define PA_D128_STAGES 2
+#ifndef PA_STAGES
+#define PA_STAGES 2
 #endif
-#ifndef PA_D64_WARPS
-#define PA_D64_WARPS 4
-#endif
-#ifndef PA_D64_STAGES
-#define PA_D64_STAGES 4
-#endif
-template <int D>
-struct Shape;
-template <>
-struct Shape<128> {
-  static constexpr int WARPS = PA_D128_WARPS, STAGES = PA_D128_STAGES;
+constexpr int kWarps = PA_WARPS, kStages = PA_STAGES;
+constexpr int kMaxSeqs = 32768;         // tile prefix kept in shared memory
+
+template <class E, int D>
+const void *split_kernel(int group) {
+  if (uses_mma(group)) return reinterpret_cast<const void *>(pa::decode_split_mma_kernel<E, D, kWarps, kStages>);
+  if (heads_per_unit(group) == 2) return reinterpret_cast<const void *>(pa::decode_split_kernel<E, D, 2, kWarps, kStages>);
+  return reinterpret_cast<const void *>(pa::decode_split_kernel<E, D, 1, kWarps, kStages>);
+}
+const void *split_kernel_for(int dtype, int head_dim, int group) {
+  if (dtype == PA_BFLOAT16) return head_dim == 128 ? split_kernel<pa::BF16, 128>(group) : split_kernel<pa::BF16, 64>(group);
+  return head_dim == 128 ? split_kernel<pa::F16, 128>(group) : split_kernel<pa::F16, 64>(group);
+}
+uint32_t split_smem(int head_dim, int group, int num_seqs) {
+  if (uses_mma(group))
+    return head_dim == 128 ? pa::MmaSmem<pa::F16, 128, kWarps, kStages>::bytes(num_seqs)
+                           : pa::MmaSmem<pa::F16, 64, kWarps, kStages>::bytes(num_seqs);
+  return head_dim == 128 ? pa::SplitSmem<kWarps, kStages, 2 * pa::TILE * 128 * 2>::bytes(num_seqs)
+                         : pa::SplitSmem<kWarps, kStages, 2 * pa::TILE * 64 * 2>::bytes(num_seqs);
+}
+
+// Resident blocks per SM of `kernel` with `smem` bytes of dynamic shared memory (cached).
+struct OccEntry {
+  int dev;
+  const void *kernel;
+  uint32_t smem;
+  int per_sm;
 };
-template <>
-struct Shape<64> {
-  static constexpr int WARPS = PA_D64_WARPS, STAGES = PA_D64_STAGES;
-};
+OccEntry g_occ[64];
+int g_occ_next = 0;
 
-#ifndef PA_MMA_WARPS
-#define PA_MMA_WARPS 4
-#endif
-#ifndef PA_MMA_STAGES
-#define PA_MMA_STAGES 2
-#endif
-constexpr int kMmaWarps = PA_MMA_WARPS, kMmaStages = PA_MMA_STAGES;
-template <int D>
-constexpr int mma_smem() {
-  return 1024 + kMmaWarps * kMmaStages * (2 * pa::TILE * D * 2 + 8);
-}
-
-template <int D>
-constexpr int partition_smem() {
-  return ((Shape<D>::WARPS * Shape<D>::STAGES * 8 + 127) / 128) * 128 +
-         Shape<D>::WARPS * Shape<D>::STAGES * 2 * pa::TILE * D * 2;
-}
-
-int warps_per_sm_estimate(int head_dim, bool mma) {
-  // resident warps per SM that the shared-memory budget of the partition kernel allows
-  const int smem = mma ? (head_dim == 128 ? mma_smem<128>() : mma_smem<64>())
-                       : (head_dim == 128 ? partition_smem<128>() : partition_smem<64>());
-  const int warps = mma ? kMmaWarps : (head_dim == 128 ? Shape<128>::WARPS : Shape<64>::WARPS);
-  const int ctas = std::max(1, (227 * 1024) / (smem + 1024));
-  return ctas * warps;
-}
-
-int resolve_partition(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                      int max_context_len, int requested, int sms) {
-  if (requested != 0) {
-    if (requested < 0 || requested % block_size != 0 || requested % pa::TILE != 0 || requested > 32 * block_size)
-      return PA_ERR_PARTITION;
-    return requested;
+int blocks_per_sm(const void *kernel, uint32_t smem, int *out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record(e);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (const auto &o : g_occ)
+      if (o.kernel == kernel && o.smem == smem && o.dev == dev) {
+        *out = o.per_sm;
+        return PA_OK;
+      }
   }
-  // Measured on B200: 16 blocks per unit suit the CUDA-core kernel, 8 the
-  // tensor-core kernel (its tiles go faster, so units must be more numerous).
-  const int group = num_q_heads / num_kv_heads;
-  const bool mma = uses_mma(group);
-  const long long base_units = (long long)num_seqs * num_kv_heads * (group / heads_per_unit(group));
-  const long long want = (long long)sms * warps_per_sm_estimate(head_dim, mma);
-  const int ctx = std::max(max_context_len, 1);
-  int part = (mma ? 8 : 16) * block_size;
-  // shrink while the (rough) number of units would not give every resident warp one
-  while (part > 2 * pa::TILE && part > block_size) {
-    const long long mean_parts = std::max(1LL, ((long long)ctx / 2 + part - 1) / part);
-    if (base_units * mean_parts >= want) break;
-    part /= 2;
-  }
-  // a context that fits one partition is never split
-  const int fit = ((ctx + block_size - 1) / block_size) * block_size;
-  if (fit <= part) part = std::max(fit, pa::TILE);
-  if (part % block_size) part = ((part + block_size - 1) / block_size) * block_size;
-  return part;
-}
-
-size_t workspace_bytes_for(int num_seqs, int num_q_heads, int head_dim, int max_context_len, int part) {
-  const long long n_part_max = std::max(1LL, ((long long)max_context_len + part - 1) / part);
-  if (n_part_max <= 1) return 0;
-  const size_t rows = (size_t)num_seqs * num_q_heads * n_part_max;
-  return rows * head_dim * sizeof(float) + rows * sizeof(float2);
+  // the kernel may later be launched with any smem up to the device's opt-in limit
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return record(e);
+  if (smem > (uint32_t)optin) return PA_ERR_SHAPE;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e != cudaSuccess) return record(e);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kWarps * 32, smem);
+  if (e != cudaSuccess) return record(e);
+  per_sm = std::max(per_sm, 1);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_occ[g_occ_next] = OccEntry{dev, kernel, smem, per_sm};
+  g_occ_next = (g_occ_next + 1) % 64;
+  *out = per_sm;
+  return PA_OK;
 }
 
 int check_decode_shape(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                        int32_t block_size, int32_t max_context_len) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0) return PA_ERR_SHAPE;
+  if (num_seqs > kMaxSeqs) return PA_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
   if (num_q_heads % num_kv_heads != 0) return PA_ERR_HEADS;
   return PA_OK;
 }
 
-template <class E, int D, int G>
-int launch_partition(const pa::DecodeArgs &args, int sms, cudaStream_t stream) {
-  constexpr int WARPS = Shape<D>::WARPS, STAGES = Shape<D>::STAGES;
-  constexpr int SMEM = partition_smem<D>();
-  auto kernel = pa::decode_partition_kernel<E, D, G, WARPS, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (e != cudaSuccess) return record(e);
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, WARPS * 32, SMEM);
-  if (e != cudaSuccess) return record(e);
-  per_sm = std::max(per_sm, 1);
-  const long long need = (args.n_slots + WARPS - 1) / WARPS;
-  const int grid = (int)std::max(1LL, std::min<long long>((long long)sms * per_sm, need));
-  kernel<<<grid, WARPS * 32, SMEM, stream>>>(args);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return record(e);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+// Grid, shared memory and workspace layout of one decode call.  The workspace
+// size does not depend on the storage type: it is sized for the larger of the
+// two instantiations' grids, and the launch never uses more warps than that.
+struct LaunchPlan {
+  uint32_t smem;
+  int grid;          // blocks of the split kernel (for `dtype`; 0 if not asked)
+  long long max_chunks;
+  int chunk_tiles;   // 0: balanced
+  size_t tiles_bytes, ml_bytes, acc_bytes, total_bytes;
+};
+
+int plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                int partition_tokens, int dtype, LaunchPlan *lp) {
+  if (partition_tokens < 0 || partition_tokens % pa::TILE != 0) return PA_ERR_PARTITION;
+  int sms = 0;
+  int rc = current_sms(&sms);
+  if (rc != PA_OK) return rc;
+  const int group = num_q_heads / num_kv_heads;
+  const int G = heads_per_unit(group);
+  lp->smem = split_smem(head_dim, group, num_seqs);
+  if (lp->smem > 227u * 1024u) return PA_ERR_SHAPE;
+  int occ_f16 = 0, occ_bf16 = 0;
+  if ((rc = blocks_per_sm(split_kernel_for(PA_FLOAT16, head_dim, group), lp->smem, &occ_f16)) != PA_OK) return rc;
+  if ((rc = blocks_per_sm(split_kernel_for(PA_BFLOAT16, head_dim, group), lp->smem, &occ_bf16)) != PA_OK) return rc;
+  const long long ws_warps = (long long)sms * std::max(occ_f16, occ_bf16) * kWarps;
+  lp->grid = dtype == 0 ? 0 : sms * (dtype == PA_BFLOAT16 ? occ_bf16 : occ_f16);
+  lp->chunk_tiles = partition_tokens / pa::TILE;
+  if (lp->chunk_tiles == 0) {
+    lp->max_chunks = ws_warps;
+  } else {
+    const long long per_seq = ((long long)max_context_len + pa::TILE - 1) / pa::TILE;
+    const long long total = (long long)num_seqs * num_kv_heads * (group / G) * per_seq;
+    lp->max_chunks = std::max(1LL, (total + lp->chunk_tiles - 1) / lp->chunk_tiles);
+  }
+  lp->tiles_bytes = (((size_t)num_seqs + 1) * sizeof(int) + 255) / 256 * 256;
+  lp->ml_bytes = (size_t)lp->max_chunks * 2 * G * sizeof(float2);
+  lp->acc_bytes = (size_t)lp->max_chunks * 2 * G * head_dim * sizeof(float);
+  lp->total_bytes = lp->tiles_bytes + lp->ml_bytes + lp->acc_bytes;
   return PA_OK;
 }
 
@@ -196,7 +200,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder(int *rc) {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
-    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   if (!fn) {
     t_last_cuda_error = err != cudaSuccess ? cudaGetErrorString(err) : "cuTensorMapEncodeTiled not available";
@@ -241,10 +246,10 @@ int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, 
   const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)pa::TILE};
   const cuuint32_t elem_strides[2] = {1, 1};
-  const CUresult r = encode(&map, dtype == PA_BFLOAT16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                            2, const_cast<void *>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r =
+      encode(&map, dtype == PA_BFLOAT16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+             const_cast<void *>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     t_last_cuda_error = "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")";
     return PA_ERR_CUDA;
@@ -256,46 +261,29 @@ int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, 
 }
 
 template <class E, int D>
-int launch_mma(const pa::DecodeArgs &args, int dtype, int sms, cudaStream_t stream) {
-  const long long rows = args.num_blocks * args.num_kv_heads * args.block_size;
-  if (rows > 0xffffffffLL) return PA_ERR_SHAPE;  // beyond what a tensor map (and the row index) can address
-  CUtensorMap mk, mv;
-  int rc = cache_tensor_map(args.k_cache, rows, D, dtype, &mk);
-  if (rc != PA_OK) return rc;
-  rc = cache_tensor_map(args.v_cache, rows, D, dtype, &mv);
-  if (rc != PA_OK) return rc;
-  constexpr int SMEM = mma_smem<D>();
-  auto kernel = pa::decode_partition_mma_kernel<E, D, kMmaWarps, kMmaStages>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (e != cudaSuccess) return record(e);
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kMmaWarps * 32, SMEM);
-  if (e != cudaSuccess) return record(e);
-  per_sm = std::max(per_sm, 1);
-  const long long need = (args.n_slots + kMmaWarps - 1) / kMmaWarps;
-  const int grid = (int)std::max(1LL, std::min<long long>((long long)sms * per_sm, need));
-  kernel<<<grid, kMmaWarps * 32, SMEM, stream>>>(mk, mv, args);
-  e = cudaGetLastError();
+int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype, int sms, cudaStream_t stream) {
+  const int threads = kWarps * 32;
+  if (uses_mma(args.group)) {
+    const long long rows = args.num_blocks * args.num_kv_heads * args.block_size;
+    if (rows > 0x7fffffffLL) return PA_ERR_SHAPE;  // TMA coordinates are signed 32-bit
+    CUtensorMap mk, mv;
+    int rc = cache_tensor_map(args.k_cache, rows, D, dtype, &mk);
+    if (rc != PA_OK) return rc;
+    rc = cache_tensor_map(args.v_cache, rows, D, dtype, &mv);
+    if (rc != PA_OK) return rc;
+    pa::decode_split_mma_kernel<E, D, kWarps, kStages><<<lp.grid, threads, lp.smem, stream>>>(mk, mv, args);
+  } else if (args.heads_per_unit == 2) {
+    pa::decode_split_kernel<E, D, 2, kWarps, kStages><<<lp.grid, threads, lp.smem, stream>>>(args);
+  } else {
+    pa::decode_split_kernel<E, D, 1, kWarps, kStages><<<lp.grid, threads, lp.smem, stream>>>(args);
+  }
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  return PA_OK;
-}
-
-template <class E, int D>
-int launch_decode_d(const pa::DecodeArgs &args, int dtype, int sms, cudaStream_t stream) {
-  int rc;
-  if (uses_mma(args.group)) {
-    rc = launch_mma<E, D>(args, dtype, sms, stream);
-  } else if (args.heads_per_unit == 2) {
-    rc = launch_partition<E, D, 2>(args, sms, stream);
-  } else {
-    rc = launch_partition<E, D, 1>(args, sms, stream);
-  }
-  if (rc != PA_OK || args.n_part_max <= 1) return rc;
   const long long warps = (long long)args.num_seqs * args.num_q_heads;
   const int grid = (int)std::max(1LL, std::min<long long>((warps + 7) / 8, (long long)sms * 8));
-  pa::decode_reduce_kernel<E, D><<<grid, 256, 0, stream>>>(args);
-  cudaError_t e = cudaGetLastError();
+  pa::decode_merge_kernel<E, D><<<grid, 256, 0, stream>>>(args);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return PA_OK;
@@ -371,30 +359,14 @@ int pa_write_kv(const void *k, const void *v, void *k_cache, void *v_cache, cons
   return PA_OK;
 }
 
-int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                                   int32_t block_size, int32_t max_context_len) {
-  int rc = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len);
-  if (rc != PA_OK) return rc;
-  int sms = 0;
-  rc = current_sms(&sms);
-  if (rc != PA_OK) return rc;
-  return resolve_partition(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, 0, sms);
-}
-
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                 int32_t block_size, int32_t max_context_len, int32_t partition_tokens) {
   if (check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len) != PA_OK)
     return 0;
-  int part = partition_tokens;
-  if (part == 0) {
-    int sms = 0;
-    if (current_sms(&sms) != PA_OK) return 0;
-    part = resolve_partition(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, 0, sms);
-  } else if (resolve_partition(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, part,
-                               1) < 0) {
+  LaunchPlan lp;
+  if (plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, 0, &lp) != PA_OK)
     return 0;
-  }
-  return workspace_bytes_for(num_seqs, num_q_heads, head_dim, max_context_len, part);
+  return lp.total_bytes;
 }
 
 int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
@@ -408,6 +380,7 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   if (num_blocks <= 0 || block_table_stride <= 0) return PA_ERR_SHAPE;
   const int64_t row = (int64_t)num_q_heads * head_dim;
   if (q_seq_stride < row || out_seq_stride < row) return PA_ERR_SHAPE;
+  if (partition_tokens < 0 || partition_tokens % pa::TILE != 0) return PA_ERR_PARTITION;
   if (num_seqs == 0) return PA_OK;
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_NULL;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || (q_seq_stride % 8) ||
@@ -417,15 +390,14 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   int sms = 0;
   rc = current_sms(&sms);
   if (rc != PA_OK) return rc;
-  const int part = resolve_partition(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
-                                     partition_tokens, sms);
-  if (part < 0) return part;
-  const int n_part_max = (int)std::max(1LL, ((long long)max_context_len + part - 1) / part);
-  const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, max_context_len, part);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
+  LaunchPlan lp;
+  rc = plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, dtype, &lp);
+  if (rc != PA_OK) return rc;
+  if (!workspace || workspace_bytes < lp.total_bytes || !aligned16(workspace)) return PA_ERR_WORKSPACE;
 
   const int group = num_q_heads / num_kv_heads;
   const int G = heads_per_unit(group);
+  char *ws = static_cast<char *>(workspace);
   pa::DecodeArgs a;
   a.q = static_cast<const uint16_t *>(q);
   a.k_cache = static_cast<const uint16_t *>(k_cache);
@@ -433,13 +405,13 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.out = static_cast<uint16_t *>(out);
-  a.ws_acc = need ? static_cast<float *>(workspace) : nullptr;
-  a.ws_ml = need ? reinterpret_cast<float2 *>(static_cast<char *>(workspace) +
-                                              (size_t)num_seqs * num_q_heads * n_part_max * head_dim * sizeof(float))
-                 : nullptr;
+  a.ws_tiles = reinterpret_cast<int *>(ws);
+  a.ws_ml = reinterpret_cast<float2 *>(ws + lp.tiles_bytes);
+  a.ws_acc = reinterpret_cast<float *>(ws + lp.tiles_bytes + lp.ml_bytes);
   a.num_blocks = num_blocks;
   a.q_seq_stride = q_seq_stride;
   a.out_seq_stride = out_seq_stride;
+  a.max_chunks = lp.max_chunks;
   a.wait_limit_ns = kWaitLimitNs;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);  // log2(e)
   a.num_seqs = num_seqs;
@@ -448,18 +420,17 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   a.block_size = block_size;
   a.table_stride = block_table_stride;
   a.max_context_len = max_context_len;
-  a.part_tokens = part;
-  a.n_part_max = n_part_max;
   a.group = group;
-  a.n_chunks = group / G;
   a.heads_per_unit = G;
-  a.n_slots = (long long)n_part_max * num_seqs * num_kv_heads * a.n_chunks;
+  a.n_chunks = group / G;
+  a.chunk_tiles = lp.chunk_tiles;
+  a.split_warps = lp.grid * kWarps;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == PA_BFLOAT16;
   if (head_dim == 128)
-    return bf16 ? launch_decode_d<pa::BF16, 128>(a, dtype, sms, st) : launch_decode_d<pa::F16, 128>(a, dtype, sms, st);
-  return bf16 ? launch_decode_d<pa::BF16, 64>(a, dtype, sms, st) : launch_decode_d<pa::F16, 64>(a, dtype, sms, st);
+    return bf16 ? launch_decode_d<pa::BF16, 128>(a, lp, dtype, sms, st) : launch_decode_d<pa::F16, 128>(a, lp, dtype, sms, st);
+  return bf16 ? launch_decode_d<pa::BF16, 64>(a, lp, dtype, sms, st) : launch_decode_d<pa::F16, 64>(a, lp, dtype, sms, st);
 }
 
 int pa_get_device_status(uint32_t *status_out, int32_t clear, void *stream) {
@@ -489,7 +460,7 @@ const char *pa_status_string(int32_t status) {
     case PA_ERR_UNSUPPORTED: return "head_dim must be 64 or 128 and block_size 16 or 32";
     case PA_ERR_HEADS: return "num_q_heads must be a multiple of num_kv_heads";
     case PA_ERR_WORKSPACE: return "workspace missing, smaller than pa_decode_workspace_size() or misaligned";
-    case PA_ERR_PARTITION: return "partition_tokens must be a multiple of block_size and of 16, at most 32 blocks";
+    case PA_ERR_PARTITION: return "partition_tokens must be 0 or a positive multiple of 16";
     case PA_ERR_CUDA: return "a CUDA runtime call failed (see pa_last_cuda_error)";
     case PA_ERR_STATIC_WORKSPACE:
       return "the problem needs more split-context scratch than the library's fixed 32 MiB array; "

@@ -117,6 +117,17 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const WriteArgs a) {
 }
 
 // ---------------------------------------------------------------- K2/K3: decode
+//
+// Work decomposition ("split over a tile stream"): every sequence s with a
+// valid, non-empty context owns nt(s) = ceil(L_s / 16) tiles per head chunk
+// (a head chunk = one kv head and up to 8 of its query heads).  All tiles are
+// laid in one stream, ordered by sequence, then head chunk, then tile, and the
+// stream is cut into equal chunks of consecutive tiles; the warps of the
+// split kernel take chunks round-robin.  With the default chunk length
+// (total tiles / warps) every warp gets the same number of tiles, whatever the
+// length mix.  The part of a chunk that falls in one (sequence, head chunk)
+// is a piece: a piece that covers its whole segment writes the final output,
+// the others write a partial softmax state that the merge kernel combines.
 struct DecodeArgs {
   const uint16_t *q;
   const uint16_t *k_cache;
@@ -124,114 +135,162 @@ struct DecodeArgs {
   const int32_t *block_tables;
   const int32_t *context_lens;
   uint16_t *out;
-  float *ws_acc;  // [S][Hq][n_part_max][D] un-normalised partial outputs
-  float2 *ws_ml;  // [S][Hq][n_part_max] (running max in log2 units, running sum)
-  long long num_blocks, q_seq_stride, out_seq_stride, n_slots;
+  int *ws_tiles;   // [num_seqs + 1] tile prefix, written by block 0 of the split kernel for the merge kernel
+  float2 *ws_ml;   // [max_chunks][2][heads_per_unit] (running max in base-2 units, running sum) of partial pieces
+  float *ws_acc;   // [max_chunks][2][heads_per_unit][head_dim] un-normalised partial outputs
+  long long num_blocks, q_seq_stride, out_seq_stride, max_chunks;
   unsigned long long wait_limit_ns;
-  float scale_log2;  // scale * log2(e): logits are kept in base-2 units
-  int num_seqs, num_q_heads, num_kv_heads, block_size, table_stride;
-  int max_context_len, part_tokens, n_part_max, group, n_chunks;
-  int heads_per_unit;  // query heads sharing one kv head handled by one unit (group / n_chunks)
+  float scale_log2;  // scale * log2(e)
+  int num_seqs, num_q_heads, num_kv_heads, block_size, table_stride, max_context_len;
+  int group;           // query heads per kv head
+  int n_chunks;        // head chunks per kv head
+  int heads_per_unit;  // query heads per head chunk (group / n_chunks)
+  int chunk_tiles;     // tiles per chunk; 0: total tiles / split_warps
+  int split_warps;     // warps in the split kernel's grid
 };
 
 __device__ __forceinline__ bool context_ok(const DecodeArgs &a, int L) {
   return L >= 0 && (long long)L <= (long long)a.table_stride * a.block_size && L <= a.max_context_len;
 }
 
-// One work unit: partition p of sequence s, kv head h, query heads
-// hq0 .. hq0 + heads_per_unit - 1.
-struct Unit {
-  int s, h, p, hq0, L, tok_begin, tok_end, blk_begin, nblk;
-  bool work;  // context valid and non-empty: tiles to stream
-};
-
-// A warp's static, strided list of unit slots.  Slot order is partition
-// index outermost, then sequence, kv head, query-head chunk; slot p of a
-// sequence is empty when p * part_tokens >= L (slot p = 0 always exists: it
-// zeroes the rows of empty or invalid sequences).
-struct UnitList {
-  long long base, nwarps, per_part, per_seq;
-  int lane;
-
-  __device__ __forceinline__ UnitList(const DecodeArgs &a, int warps_per_block) {
-    lane = threadIdx.x & 31;
-    nwarps = (long long)gridDim.x * warps_per_block;
-    per_seq = (long long)a.num_kv_heads * a.n_chunks;
-    per_part = (long long)a.num_seqs * per_seq;
-    base = (long long)blockIdx.x * warps_per_block + (threadIdx.x >> 5);
-  }
-
-  // Next non-empty slot (32 candidates per step, one per lane); -1 when none is left.
-  __device__ __forceinline__ long long next(const DecodeArgs &a, int &L_out) {
-    while (base < a.n_slots) {
-      const long long c = base + (long long)lane * nwarps;
-      bool live = false;
-      int Lc = 0;
-      if (c < a.n_slots) {
-        const int p = (int)(c / per_part);
-        const int s = (int)((c - (long long)p * per_part) / per_seq);
-        Lc = __ldg(a.context_lens + s);
-        live = (p == 0) || (context_ok(a, Lc) && (long long)p * a.part_tokens < Lc);
-      }
-      const unsigned m = __ballot_sync(FULL, live);
-      if (m) {
-        const int idx = __ffs(m) - 1;
-        L_out = __shfl_sync(FULL, Lc, idx);
-        const long long slot = base + (long long)idx * nwarps;
-        base = slot + nwarps;
-        return slot;
-      }
-      base += 32LL * nwarps;
-    }
-    return -1;
-  }
-
-  __device__ __forceinline__ Unit describe(const DecodeArgs &a, long long slot, int L) const {
-    Unit u;
-    u.p = (int)(slot / per_part);
-    long long rem = slot - (long long)u.p * per_part;
-    u.s = (int)(rem / per_seq);
-    rem -= (long long)u.s * per_seq;
-    u.h = (int)(rem / a.n_chunks);
-    u.hq0 = u.h * a.group + (int)(rem - (long long)u.h * a.n_chunks) * a.heads_per_unit;
-    u.L = L;
-    u.work = context_ok(a, L) && L > 0;
-    u.tok_begin = u.p * a.part_tokens;
-    u.tok_end = u.work ? min(L, u.tok_begin + a.part_tokens) : u.tok_begin;
-    u.blk_begin = u.tok_begin / a.block_size;
-    u.nblk = (u.tok_end - u.tok_begin + a.block_size - 1) / a.block_size;  // <= 32
-    return u;
-  }
-};
-
-// The unit's table entry for this lane (block blk_begin + lane), or 0.
-__device__ __forceinline__ int unit_table_entry(const DecodeArgs &a, const Unit &u, int lane) {
-  return (u.work && lane < u.nblk) ? __ldg(a.block_tables + (long long)u.s * a.table_stride + u.blk_begin + lane) : 0;
+__device__ __forceinline__ int seq_tiles(const DecodeArgs &a, int L) {
+  return (context_ok(a, L) && L > 0) ? (L + TILE - 1) / TILE : 0;
 }
 
-// Status bits and zero rows for a unit that streams nothing (empty or invalid
-// context, or a table entry outside the pool).
-__device__ __forceinline__ void unit_without_tiles(const DecodeArgs &a, const Unit &u, bool bad_entry, int lane,
-                                                   int D) {
-  const int n_parts = u.work ? (u.L + a.part_tokens - 1) / a.part_tokens : 1;
-  if (lane == 0) {
-    if (!u.work && u.L != 0)
-      atomicOr(&g_status, (u.L < 0 || (long long)u.L > (long long)a.table_stride * a.block_size)
-                              ? PA_DEV_ERR_CONTEXT
-                              : PA_DEV_ERR_CONTEXT_HINT);
-    if (u.work && bad_entry) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
+// pt[s] = tiles (per head chunk) of the sequences before s, s = 0..num_seqs.
+// Called by every thread of the block; ends with a block barrier.
+// `scratch` holds one int per warp.
+__device__ __forceinline__ void build_tile_prefix(const DecodeArgs &a, int *pt, int *scratch) {
+  const int S = a.num_seqs;
+  const int nth = blockDim.x, tid = threadIdx.x;
+  const int per = (S + nth - 1) / nth;
+  const int i0 = min(S, tid * per), i1 = min(S, i0 + per);
+  int sum = 0;
+  for (int i = i0; i < i1; ++i) {
+    const int nt = seq_tiles(a, __ldg(a.context_lens + i));
+    pt[i + 1] = nt;
+    sum += nt;
   }
-  if (n_parts == 1) {
-    for (int i = lane; i < a.heads_per_unit * D / 8; i += 32) {
-      const int gg = i / (D / 8), c = i - gg * (D / 8);
-      *reinterpret_cast<uint4 *>(a.out + (long long)u.s * a.out_seq_stride + (long long)(u.hq0 + gg) * D + c * 8) =
-          make_uint4(0, 0, 0, 0);
-    }
-  } else if (lane < a.heads_per_unit) {
-    // a partial marked invalid: the merge kernel zeroes the row
-    a.ws_ml[((long long)u.s * a.num_q_heads + u.hq0 + lane) * a.n_part_max + u.p] = make_float2(-INFINITY, -1.f);
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(FULL, incl, off);
+    if (lane >= off) incl += y;
   }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int run = incl - sum;
+  for (int w = 0; w < warp; ++w) run += scratch[w];
+  for (int i = i0; i < i1; ++i) {
+    run += pt[i + 1];
+    pt[i + 1] = run;
+  }
+  if (tid == 0) pt[0] = 0;
+  __syncthreads();
 }
+
+constexpr int MIN_AUTO_CHUNK_TILES = 4;  // the balanced split never cuts finer than this
+
+struct ChunkPlan {
+  long long total, chunk, count;
+};
+
+// Chunk length and count for a tile stream of pt[S] * head_chunks tiles.
+__device__ __forceinline__ ChunkPlan plan_chunks(const DecodeArgs &a, int tiles_per_chunk_set) {
+  ChunkPlan p;
+  p.total = (long long)tiles_per_chunk_set * a.num_kv_heads * a.n_chunks;
+  long long c = a.chunk_tiles > 0 ? a.chunk_tiles
+                                  : max((p.total + a.split_warps - 1) / a.split_warps, (long long)MIN_AUTO_CHUNK_TILES);
+  c = max(c, (p.total + a.max_chunks - 1) / a.max_chunks);  // never more chunks than the workspace holds
+  p.chunk = max(c, 1LL);
+  p.count = (p.total + p.chunk - 1) / p.chunk;
+  return p;
+}
+
+// A position in the tile stream: tile j of head chunk hc of sequence s (nt tiles).
+struct TilePos {
+  int s, hc, j, nt;
+};
+
+__device__ __forceinline__ TilePos locate_tile(const int *pt, int S, int HC, long long t) {
+  int lo = 0, hi = S - 1;  // largest s with pt[s] * HC <= t; that sequence has tiles
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)pt[mid] * HC <= t)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  TilePos p;
+  p.s = lo;
+  p.nt = pt[lo + 1] - pt[lo];
+  const long long r = t - (long long)pt[lo] * HC;
+  p.hc = (int)(r / p.nt);
+  p.j = (int)(r - (long long)p.hc * p.nt);
+  return p;
+}
+
+__device__ __forceinline__ void advance_tile(TilePos &p, const int *pt, int S, int HC) {
+  if (++p.j < p.nt) return;
+  p.j = 0;
+  if (++p.hc < HC) return;
+  p.hc = 0;
+  do {
+    ++p.s;
+  } while (p.s < S && pt[p.s + 1] == pt[p.s]);
+  p.nt = p.s < S ? pt[p.s + 1] - pt[p.s] : 0;
+}
+
+// First query head of head chunk hc (kv head hc / n_chunks).
+__device__ __forceinline__ int chunk_first_head(const DecodeArgs &a, int hc) {
+  const int h = hc / a.n_chunks;
+  return h * a.group + (hc - h * a.n_chunks) * a.heads_per_unit;
+}
+
+// The copy side of a warp's tile stream: walks the chunk ahead of the
+// consumer, looks the physical block of each tile up in a 32-entry window of
+// the sequence's table (one entry per lane), and starts the copies of the
+// tile into a ring slot.  A tile whose table entry lies outside the pool is
+// not copied: its slot's barrier is completed with a plain arrive and the
+// slot is flagged in `bad_slots`.
+struct TileProducer {
+  TilePos pos;
+  int win_s, win_base, win_nblk, ent;
+  uint32_t bad_slots;
+
+  __device__ __forceinline__ void start(const TilePos &p) {
+    pos = p;
+    win_s = -1;
+    win_base = 0;
+    win_nblk = 0;
+    ent = -1;
+    bad_slots = 0;
+  }
+
+  // Returns the physical block of the producer's current tile (or -1), loading a new window when needed.
+  __device__ __forceinline__ int lookup(const DecodeArgs &a, int lane) {
+    const int blk = (pos.j * TILE) / a.block_size;
+    if (pos.s != win_s || blk < win_base || blk >= win_base + 32) {
+      if (pos.s != win_s) {
+        win_s = pos.s;
+        const int L = __ldg(a.context_lens + pos.s);
+        win_nblk = (L + a.block_size - 1) / a.block_size;
+      }
+      win_base = blk & ~31;
+      ent = (win_base + lane < win_nblk)
+                ? __ldg(a.block_tables + (long long)pos.s * a.table_stride + win_base + lane)
+                : -1;
+    }
+    const int phys = __shfl_sync(FULL, ent, blk - win_base);
+    return (phys >= 0 && (long long)phys < a.num_blocks) ? phys : -1;
+  }
+
+  // Global row (in [num_blocks * num_kv_heads * block_size)) of the tile's first token.
+  __device__ __forceinline__ long long first_row(const DecodeArgs &a, int phys) const {
+    return ((long long)phys * a.num_kv_heads + pos.hc / a.n_chunks) * a.block_size + (pos.j * TILE) % a.block_size;
+  }
+};
 
 // Sums, over the lanes of one row group (lane bits 0..log2(2R)-1), R partial
 // dot products held by every lane, with R/2 + R/4 + ... + 1 + 1 shuffles
@@ -281,152 +340,156 @@ __device__ __forceinline__ float dot8_bf16(const uint32_t (&q)[4], const uint4 k
   return d;
 }
 
-// Each warp is an independent worker: it walks its own static, strided list
-// of work units (UnitList) and streams each unit's 16-token K/V tiles through
-// a private STAGES-deep ring of shared-memory buffers filled by bulk copies.
-// There is no block-level barrier.  Used for groups of G <= 2 query heads per
-// kv head (CUDA cores).
+// Shared-memory layout of the split kernels: [ring slots][per-warp barriers][tile prefix][scan scratch].
+template <int WARPS, int STAGES, uint32_t STAGE_BYTES>
+struct SplitSmem {
+  static constexpr uint32_t RING = WARPS * STAGES * STAGE_BYTES;
+  static constexpr uint32_t BARS = ((WARPS * STAGES * 8 + 127) / 128) * 128;
+  static __host__ __device__ constexpr uint32_t bytes(int num_seqs) {
+    return RING + BARS + (uint32_t)(num_seqs + 1 + WARPS) * 4u;
+  }
+};
+
+// Waits (bounded) for ring slot `it`; on a timeout flags the status, lets the
+// copies still in flight land (bounded) and returns false.
+template <int STAGES>
+__device__ __forceinline__ bool wait_slot(uint64_t *bars, uint32_t it, int in_flight, unsigned long long limit_ns,
+                                          int lane) {
+  const bool arrived = mbar_wait_bounded(&bars[it % STAGES], (it / STAGES) & 1u, limit_ns);
+  if (!__any_sync(FULL, !arrived)) return true;
+  if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
+  for (int k = 0; k < in_flight; ++k) {
+    const uint32_t i2 = it + k;
+    mbar_wait_bounded(&bars[i2 % STAGES], (i2 / STAGES) & 1u, limit_ns);
+  }
+  return false;
+}
+
+// CUDA-core split kernel, for head chunks of G = 1 or 2 query heads.
 //
-// Per tile, lane l copies 16 bytes (8 head dims) of rows r*NGRP + l/LPR
-// (r < R) of K and of V from the ring into registers, and the ring slot is
-// refilled at once, before any arithmetic, so the copies in flight never wait
-// on the math.  The next unit's table entries and query rows are loaded while
-// the current unit runs.  QK^T uses the mixed-precision fma (2-byte inputs,
-// fp32 accumulation); the 16 dot products are finished by a reduce-scatter
-// butterfly.  The online softmax keeps, per query head, a running maximum m
-// that is raised only when a logit exceeds it by more than RESCALE_SLACK
-// (base-2 units), so most tiles need no max reduction; m cancels between the
-// numerator and the denominator, and the weights stay below 2^RESCALE_SLACK.
+// Each warp streams the tiles of its chunks through a private STAGES-deep ring
+// of shared-memory slots filled by bulk copies (K tile + V tile of one
+// (block, kv head), 2 x 16 * D * 2 bytes).  Per tile, lane l copies 16 bytes
+// (8 head dims) of rows r*NGRP + l/LPR (r < R) of K and of V from the slot
+// into registers and the slot is refilled at once, before the math.  QK^T uses
+// the mixed-precision fma (2-byte inputs, fp32 accumulation); the 16 dot
+// products are finished by a reduce-scatter butterfly.  The online softmax
+// keeps, per query head, a running maximum m that is raised only when a logit
+// exceeds it by more than RESCALE_SLACK (base-2 units), so most tiles need no
+// max reduction; m cancels between numerator and denominator, and weights
+// stay below 2^RESCALE_SLACK.
 constexpr float RESCALE_SLACK = 8.f;
 
 template <class E, int D, int G, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32) decode_partition_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeArgs a) {
   constexpr int LPR = D / 8;       // lanes covering one K/V row
   constexpr int NGRP = 32 / LPR;   // rows one warp-wide 16-byte load covers
   constexpr int R = TILE / NGRP;   // rows per lane per tile
   constexpr uint32_t TILE_BYTES = TILE * D * 2;
   constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;
-  constexpr int BAR_BYTES = ((WARPS * STAGES * 8 + 127) / 128) * 128;
+  using Smem = SplitSmem<WARPS, STAGES, STAGE_BYTES>;
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem) + warp * STAGES;
-  unsigned char *ring = smem + BAR_BYTES + warp * STAGES * STAGE_BYTES;
+  unsigned char *ring = smem + warp * STAGES * STAGE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Smem::RING) + warp * STAGES;
+  int *pt = reinterpret_cast<int *>(smem + Smem::RING + Smem::BARS);
   if (lane == 0) {
 #pragma unroll
     for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
   }
-  __syncwarp();
+  const int S = a.num_seqs;
+  build_tile_prefix(a, pt, pt + S + 1);
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i <= S; i += blockDim.x) a.ws_tiles[i] = pt[i];
+  const ChunkPlan plan = plan_chunks(a, pt[S]);
+  const int HC = a.num_kv_heads * a.n_chunks;
 
   const int grp = lane / LPR;
   const int cl = lane % LPR;
   const int my_tok = ((lane & (LPR - 2)) >> 1) * NGRP + grp;  // token whose logit this lane ends with
-  uint32_t iter = 0;  // tiles consumed by this warp so far: ring slot iter % STAGES, phase (iter / STAGES) & 1
+  uint32_t iter = 0;  // tiles consumed by this warp: ring slot iter % STAGES, phase (iter / STAGES) & 1
+  TileProducer prod;
 
-  UnitList list(a, WARPS);
-  auto fetch_q = [&](const Unit &u, uint4 (&qraw)[G]) {
-#pragma unroll
-    for (int gg = 0; gg < G; ++gg)
-      qraw[gg] = u.work ? __ldg(reinterpret_cast<const uint4 *>(a.q + (long long)u.s * a.q_seq_stride +
-                                                                (long long)(u.hq0 + gg) * D + cl * 8))
-                        : make_uint4(0, 0, 0, 0);
-  };
+  for (long long c = (long long)blockIdx.x * WARPS + warp; c < plan.count; c += (long long)gridDim.x * WARPS) {
+    const long long t0 = c * plan.chunk;
+    const int ntile = (int)min(plan.chunk, plan.total - t0);
+    TilePos cp = locate_tile(pt, S, HC, t0);
+    prod.start(cp);
 
-  int L0 = 0;
-  const long long first = list.next(a, L0);
-  if (first < 0) return;
-  Unit cur = list.describe(a, first, L0);
-  int ent = unit_table_entry(a, cur, lane);
-  uint4 qraw[G];
-  fetch_q(cur, qraw);
-
-  while (true) {
-    const int n_parts = cur.work ? (cur.L + a.part_tokens - 1) / a.part_tokens : 1;
-    const int ntiles = (cur.tok_end - cur.tok_begin + TILE - 1) / TILE;
-    const bool bad = __any_sync(FULL, cur.work && lane < cur.nblk && (ent < 0 || (long long)ent >= a.num_blocks));
-
-    // ---- issue one tile: K and V rows [tok0, tok0 + 16) of (block, h) into ring slot it % STAGES
-    auto issue = [&](int j, uint32_t it) {
-      const int tok0 = cur.tok_begin + j * TILE;
-      const int phys = __shfl_sync(FULL, ent, tok0 / a.block_size - cur.blk_begin);
+    auto issue_next = [&](uint32_t it) {
+      const int phys = prod.lookup(a, lane);
+      const int st = (int)(it % STAGES);
+      prod.bad_slots = phys >= 0 ? (prod.bad_slots & ~(1u << st)) : (prod.bad_slots | (1u << st));
       if (lane == 0) {
-        const int st = (int)(it % STAGES);
-        const long long row0 = ((long long)phys * a.num_kv_heads + cur.h) * a.block_size + (tok0 % a.block_size);
-        unsigned char *dst = ring + st * STAGE_BYTES;
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
-        bulk_copy_g2s(dst, a.k_cache + row0 * D, TILE_BYTES, &bars[st]);
-        bulk_copy_g2s(dst + TILE_BYTES, a.v_cache + row0 * D, TILE_BYTES, &bars[st]);
+        if (phys >= 0) {
+          const long long row0 = prod.first_row(a, phys);
+          unsigned char *dst = ring + st * STAGE_BYTES;
+          mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
+          bulk_copy_g2s(dst, a.k_cache + row0 * D, TILE_BYTES, &bars[st]);
+          bulk_copy_g2s(dst + TILE_BYTES, a.v_cache + row0 * D, TILE_BYTES, &bars[st]);
+        } else {
+          mbar_arrive(&bars[st]);
+        }
       }
+      advance_tile(prod.pos, pt, S, HC);
     };
-    const int npro = (cur.work && !bad) ? min(ntiles, STAGES) : 0;
-    for (int j = 0; j < npro; ++j) issue(j, iter + j);
+    const int npro = min(ntile, STAGES);
+    for (int k = 0; k < npro; ++k) issue_next(iter + k);
 
-    // ---- look up and prefetch the next unit while those copies are in flight
-    int Ln = 0;
-    const long long nslot = list.next(a, Ln);
-    Unit nxt = cur;
-    int ent_n = 0;
-    uint4 qraw_n[G];
-    if (nslot >= 0) {
-      nxt = list.describe(a, nslot, Ln);
-      ent_n = unit_table_entry(a, nxt, lane);
-      fetch_q(nxt, qraw_n);
-    }
+    uint32_t qw[G][4];
+    float m[G], lsum[G];
+    float2 acc[G][4];
+    int L = 0, hq0 = 0, slot = 0;
+    bool full = false, piece_bad = false;
 
-    if (!cur.work || bad) {
-      unit_without_tiles(a, cur, bad, lane, D);
-    } else {
-      uint16_t *out_row = a.out + (long long)cur.s * a.out_seq_stride + (long long)cur.hq0 * D + cl * 8;
-      uint32_t qw[G][4];
+    for (int k = 0; k < ntile; ++k) {
+      if (k == 0 || cp.j == 0) {  // a new piece: segment (cp.s, cp.hc) from tile cp.j on
+        const int len = min(cp.nt - cp.j, ntile - k);
+        full = (cp.j == 0 && len == cp.nt);
+        slot = (k == 0) ? 0 : 1;
+        hq0 = chunk_first_head(a, cp.hc);
+        L = __ldg(a.context_lens + cp.s);
+        piece_bad = false;
 #pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        qw[gg][0] = qraw[gg].x;
-        qw[gg][1] = qraw[gg].y;
-        qw[gg][2] = qraw[gg].z;
-        qw[gg][3] = qraw[gg].w;
-      }
-      float m[G], lsum[G];
-      float2 acc[G][4];
+        for (int gg = 0; gg < G; ++gg) {
+          const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.q + (long long)cp.s * a.q_seq_stride +
+                                                                (long long)(hq0 + gg) * D + cl * 8));
+          qw[gg][0] = w.x;
+          qw[gg][1] = w.y;
+          qw[gg][2] = w.z;
+          qw[gg][3] = w.w;
+          m[gg] = -INFINITY;
+          lsum[gg] = 0.f;
 #pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        m[gg] = -INFINITY;
-        lsum[gg] = 0.f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[gg][k] = make_float2(0.f, 0.f);
-      }
-
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = (int)(iter % STAGES);
-        const uint32_t parity = (iter / STAGES) & 1u;
-        const bool arrived = mbar_wait_bounded(&bars[st], parity, a.wait_limit_ns);
-        if (__any_sync(FULL, !arrived)) {
-          // A copy never landed: report, let every copy still in flight finish (bounded), stop.
-          if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
-          const int last = min(ntiles, j + STAGES);
-          for (int jj = j; jj < last; ++jj) {
-            const uint32_t it = iter + (jj - j);
-            mbar_wait_bounded(&bars[it % STAGES], (it / STAGES) & 1u, a.wait_limit_ns);
-          }
-          return;
+          for (int kk = 0; kk < 4; ++kk) acc[gg][kk] = make_float2(0.f, 0.f);
         }
-        // copy this lane's rows out of the ring, then hand the slot straight back to the copy engine
-        const unsigned char *kt = ring + st * STAGE_BYTES;
-        const unsigned char *vt = kt + TILE_BYTES;
-        uint4 kr[R], vr[R];
+      }
+      const int st = (int)(iter % STAGES);
+      if (!wait_slot<STAGES>(bars, iter, min(STAGES, ntile - k), a.wait_limit_ns, lane)) return;
+      const bool tile_bad = (prod.bad_slots >> st) & 1u;
+      // copy this lane's rows out of the slot, then hand the slot straight back to the copy engine
+      const unsigned char *kt = ring + st * STAGE_BYTES;
+      const unsigned char *vt = kt + TILE_BYTES;
+      uint4 kr[R], vr[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          kr[r] = *reinterpret_cast<const uint4 *>(kt + ((r * NGRP + grp) * D + cl * 8) * 2);
-          vr[r] = *reinterpret_cast<const uint4 *>(vt + ((r * NGRP + grp) * D + cl * 8) * 2);
-        }
-        __syncwarp();
-        if (j + STAGES < ntiles) issue(j + STAGES, iter + STAGES);
-        ++iter;
-        const int nvalid = min(TILE, cur.tok_end - (cur.tok_begin + j * TILE));
+      for (int r = 0; r < R; ++r) {
+        kr[r] = tile_bad ? make_uint4(0, 0, 0, 0)
+                         : *reinterpret_cast<const uint4 *>(kt + ((r * NGRP + grp) * D + cl * 8) * 2);
+        vr[r] = tile_bad ? make_uint4(0, 0, 0, 0)
+                         : *reinterpret_cast<const uint4 *>(vt + ((r * NGRP + grp) * D + cl * 8) * 2);
+      }
+      __syncwarp();
+      if (k + STAGES < ntile) issue_next(iter + STAGES);
+      ++iter;
+      piece_bad |= tile_bad;
+
+      if (!piece_bad) {
+        const int nvalid = min(TILE, L - cp.j * TILE);
         const bool tok_live = my_tok < nvalid;
-
         // QK^T for this lane's R rows, the butterfly, scale, mask
         float z[G];
 #pragma unroll
@@ -447,9 +510,9 @@ __global__ void __launch_bounds__(WARPS * 32) decode_partition_kernel(const Deco
             mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 4));
             mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
             mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
-            const float alpha = exp2f(m[gg] - mt);  // 0 on the first tile (m = -inf)
+            const float alpha = exp2f(m[gg] - mt);  // 0 on the piece's first tile (m = -inf)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[gg][k] = make_float2(acc[gg][k].x * alpha, acc[gg][k].y * alpha);
+            for (int kk = 0; kk < 4; ++kk) acc[gg][kk] = make_float2(acc[gg][kk].x * alpha, acc[gg][kk].y * alpha);
             lsum[gg] *= alpha;
             m[gg] = mt;
           }
@@ -466,121 +529,139 @@ __global__ void __launch_bounds__(WARPS * 32) decode_partition_kernel(const Deco
           if (nvalid < TILE) {  // rows past the sequence may hold anything (NaN): never let them in
             const bool row_live = (r * NGRP + grp) < nvalid;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) vf[k] = row_live ? vf[k] : 0.f;
+            for (int kk = 0; kk < 8; ++kk) vf[kk] = row_live ? vf[kk] : 0.f;
           }
 #pragma unroll
           for (int gg = 0; gg < G; ++gg) {
             const float2 pp = make_float2(pr[gg][r], pr[gg][r]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[gg][k] = __ffma2_rn(pp, make_float2(vf[2 * k], vf[2 * k + 1]), acc[gg][k]);
+            for (int kk = 0; kk < 4; ++kk)
+              acc[gg][kk] = __ffma2_rn(pp, make_float2(vf[2 * kk], vf[2 * kk + 1]), acc[gg][kk]);
           }
         }
       }
 
-      // ---- merge the row groups, total the running sums, store
-#pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-#pragma unroll
-        for (int off = LPR; off < 32; off <<= 1) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            acc[gg][k].x += __shfl_xor_sync(FULL, acc[gg][k].x, off);
-            acc[gg][k].y += __shfl_xor_sync(FULL, acc[gg][k].y, off);
-          }
-        }
-        float l = lsum[gg];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
-        lsum[gg] = l;
-      }
-      if (n_parts == 1) {
-        if (lane < LPR) {
-#pragma unroll
-          for (int gg = 0; gg < G; ++gg) {
-            float o[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              o[2 * k] = acc[gg][k].x / lsum[gg];
-              o[2 * k + 1] = acc[gg][k].y / lsum[gg];
-            }
-            *reinterpret_cast<uint4 *>(out_row + gg * D) = narrow8<E>(o);
-          }
-        }
-      } else {
+      if (cp.j + 1 == cp.nt || k + 1 == ntile) {
+        // ---- end of the piece: merge the row groups, total the sums, store the output or the partial
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
-          const long long prow = ((long long)cur.s * a.num_q_heads + cur.hq0 + gg) * a.n_part_max + cur.p;
-          if (lane < LPR) {
-            float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + prow * D + cl * 8);
-            dst[0] = make_float4(acc[gg][0].x, acc[gg][0].y, acc[gg][1].x, acc[gg][1].y);
-            dst[1] = make_float4(acc[gg][2].x, acc[gg][2].y, acc[gg][3].x, acc[gg][3].y);
+#pragma unroll
+          for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              acc[gg][kk].x += __shfl_xor_sync(FULL, acc[gg][kk].x, off);
+              acc[gg][kk].y += __shfl_xor_sync(FULL, acc[gg][kk].y, off);
+            }
           }
-          if (lane == 0) a.ws_ml[prow] = make_float2(m[gg], lsum[gg]);
+          float l = lsum[gg];
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
+          lsum[gg] = l;
+        }
+        if (piece_bad && lane == 0) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
+        if (full) {
+          if (lane < LPR) {
+            uint16_t *out_row = a.out + (long long)cp.s * a.out_seq_stride + (long long)hq0 * D + cl * 8;
+#pragma unroll
+            for (int gg = 0; gg < G; ++gg) {
+              float o[8];
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                o[2 * kk] = piece_bad ? 0.f : acc[gg][kk].x / lsum[gg];
+                o[2 * kk + 1] = piece_bad ? 0.f : acc[gg][kk].y / lsum[gg];
+              }
+              *reinterpret_cast<uint4 *>(out_row + gg * D) = narrow8<E>(o);
+            }
+          }
+        } else {
+          const long long prow = (c * 2 + slot) * G;
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg) {
+            if (lane < LPR && !piece_bad) {
+              float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + (prow + gg) * D + cl * 8);
+              dst[0] = make_float4(acc[gg][0].x, acc[gg][0].y, acc[gg][1].x, acc[gg][1].y);
+              dst[1] = make_float4(acc[gg][2].x, acc[gg][2].y, acc[gg][3].x, acc[gg][3].y);
+            }
+            if (lane == 0) a.ws_ml[prow + gg] = piece_bad ? make_float2(-INFINITY, -1.f) : make_float2(m[gg], lsum[gg]);
+          }
         }
       }
+      advance_tile(cp, pt, S, HC);
     }
-
-    if (nslot < 0) break;
-    cur = nxt;
-    ent = ent_n;
-#pragma unroll
-    for (int gg = 0; gg < G; ++gg) qraw[gg] = qraw_n[gg];
   }
 }
 
-// One warp per (sequence, query head) whose context spans more than one
-// partition: out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p with
-// M = max_p m_p, in increasing p order (deterministic).
+// One warp per (sequence, query head): writes the zero rows of empty or
+// invalid sequences (setting the status bits of the invalid ones) and merges
+// the partial pieces of segments that the split kernel cut across chunks:
+// out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p, M = max_p m_p, in
+// increasing chunk order (deterministic).
 template <class E, int D>
-__global__ void __launch_bounds__(256) decode_reduce_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
   constexpr int DPL = D / 32;  // dims per lane (4 or 2)
   const int lane = threadIdx.x & 31;
-  const long long total = (long long)a.num_seqs * a.num_q_heads;
+  const int S = a.num_seqs;
+  const ChunkPlan plan = plan_chunks(a, a.ws_tiles[S]);
+  const int HC = a.num_kv_heads * a.n_chunks;
+  const long long total = (long long)S * a.num_q_heads;
   const long long nw = (long long)gridDim.x * (blockDim.x / 32);
   for (long long w = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); w < total; w += nw) {
     const int s = (int)(w / a.num_q_heads);
+    const int hq = (int)(w - (long long)s * a.num_q_heads);
     const int L = __ldg(a.context_lens + s);
-    if (L <= 0 || !context_ok(a, L)) continue;
-    const int n = (L + a.part_tokens - 1) / a.part_tokens;
-    if (n <= 1) continue;
-    const long long row0 = w * a.n_part_max;
-    float M = -INFINITY;
-    bool err = false;
-    for (int p = lane; p < n; p += 32) {
-      const float2 ml = a.ws_ml[row0 + p];
-      M = fmaxf(M, ml.x);
-      err |= ml.y < 0.f;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
-    err = __any_sync(FULL, err);
+    uint16_t *dst = a.out + (long long)s * a.out_seq_stride + (long long)hq * D + lane * DPL;
     float o[DPL];
 #pragma unroll
     for (int k = 0; k < DPL; ++k) o[k] = 0.f;
-    if (!err) {
-      float l = 0.f;
-#pragma unroll 4
-      for (int p = 0; p < n; ++p) {
-        const float2 ml = a.ws_ml[row0 + p];
-        const float wgt = exp2f(ml.x - M);
-        l = fmaf(ml.y, wgt, l);
-        const float *src = a.ws_acc + (row0 + p) * D + lane * DPL;
-        float v[DPL];
-        if constexpr (DPL == 4) {
-          const float4 t = *reinterpret_cast<const float4 *>(src);
-          v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-        } else {
-          const float2 t = *reinterpret_cast<const float2 *>(src);
-          v[0] = t.x; v[1] = t.y;
-        }
-#pragma unroll
-        for (int k = 0; k < DPL; ++k) o[k] = fmaf(wgt, v[k], o[k]);
+    if (!context_ok(a, L) || L == 0) {
+      if (lane == 0 && L != 0)
+        atomicOr(&g_status, (L < 0 || (long long)L > (long long)a.table_stride * a.block_size)
+                                ? PA_DEV_ERR_CONTEXT
+                                : PA_DEV_ERR_CONTEXT_HINT);
+    } else {
+      const int h = hq / a.group;
+      const int r = hq - h * a.group;
+      const int ch = r / a.heads_per_unit;
+      const int gg = r - ch * a.heads_per_unit;
+      const int nt = a.ws_tiles[s + 1] - a.ws_tiles[s];
+      const long long seg0 = (long long)a.ws_tiles[s] * HC + (long long)(h * a.n_chunks + ch) * nt;
+      const long long c_first = seg0 / plan.chunk, c_last = (seg0 + nt - 1) / plan.chunk;
+      if (c_first == c_last) continue;  // one chunk held the whole segment: the split kernel wrote the row
+      float M = -INFINITY;
+      bool err = false;
+      for (long long c = c_first + lane; c <= c_last; c += 32) {
+        const int slot = (c == c_first && seg0 > c * plan.chunk) ? 1 : 0;
+        const float2 ml = a.ws_ml[(c * 2 + slot) * a.heads_per_unit + gg];
+        M = fmaxf(M, ml.x);
+        err |= ml.y < 0.f;
       }
 #pragma unroll
-      for (int k = 0; k < DPL; ++k) o[k] = o[k] / l;
+      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+      err = __any_sync(FULL, err);
+      if (!err) {
+        float l = 0.f;
+        for (long long c = c_first; c <= c_last; ++c) {
+          const int slot = (c == c_first && seg0 > c * plan.chunk) ? 1 : 0;
+          const long long row = (c * 2 + slot) * a.heads_per_unit + gg;
+          const float2 ml = a.ws_ml[row];
+          const float wgt = exp2f(ml.x - M);
+          l = fmaf(ml.y, wgt, l);
+          const float *src = a.ws_acc + row * D + lane * DPL;
+          float v[DPL];
+          if constexpr (DPL == 4) {
+            const float4 t = *reinterpret_cast<const float4 *>(src);
+            v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+          } else {
+            const float2 t = *reinterpret_cast<const float2 *>(src);
+            v[0] = t.x; v[1] = t.y;
+          }
+#pragma unroll
+          for (int k = 0; k < DPL; ++k) o[k] = fmaf(wgt, v[k], o[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) o[k] = o[k] / l;
+      }
     }
-    uint16_t *dst = a.out + (long long)s * a.out_seq_stride + (long long)(w - (long long)s * a.num_q_heads) * D +
-                    lane * DPL;
     if constexpr (DPL == 4) {
       *reinterpret_cast<uint2 *>(dst) = make_uint2(E::narrow2(o[0], o[1]), E::narrow2(o[2], o[3]));
     } else {

@@ -66,13 +66,24 @@ __device__ __forceinline__ uint32_t swizzled(int r, int c) {
 }
 
 template <class E, int D, int WARPS, int STAGES>
+struct MmaSmem {
+  static constexpr uint32_t STAGE_BYTES = 2 * TILE * D * 2;
+  static constexpr uint32_t RING = WARPS * STAGES * STAGE_BYTES;
+  static constexpr uint32_t BARS = ((WARPS * STAGES * 8 + 127) / 128) * 128;
+  static __host__ __device__ constexpr uint32_t bytes(int num_seqs) {
+    return 1024 + RING + BARS + (uint32_t)(num_seqs + 1 + WARPS) * 4u;  // 1024: alignment slack
+  }
+};
+
+template <class E, int D, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32)
-    decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-                                const DecodeArgs a) {
+    decode_split_mma_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                            const DecodeArgs a) {
   constexpr int KSTEPS = D / 16;  // 16-dim steps of QK^T, and 16-dim row tiles of O^T
   constexpr int BOXES = D / 64;
   constexpr uint32_t TILE_BYTES = TILE * D * 2;
-  constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;
+  using Smem = MmaSmem<E, D, WARPS, STAGES>;
+  constexpr uint32_t STAGE_BYTES = Smem::STAGE_BYTES;
 
   extern __shared__ unsigned char smem_raw[];
   // ring slots start on a 1024-byte boundary (the swizzle pattern repeats every 1024 bytes)
@@ -80,7 +91,8 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   unsigned char *ring = smem + warp * STAGES * STAGE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + WARPS * STAGES * STAGE_BYTES) + warp * STAGES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Smem::RING) + warp * STAGES;
+  int *pt = reinterpret_cast<int *>(smem + Smem::RING + Smem::BARS);
   if (lane == 0) {
 #pragma unroll
     for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
@@ -88,7 +100,13 @@ __global__ void __launch_bounds__(WARPS * 32)
     prefetch_tensor_map(&tmap_k);
     prefetch_tensor_map(&tmap_v);
   }
-  __syncwarp();
+  const int S = a.num_seqs;
+  build_tile_prefix(a, pt, pt + S + 1);
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i <= S; i += blockDim.x) a.ws_tiles[i] = pt[i];
+  const ChunkPlan plan = plan_chunks(a, pt[S]);
+  const int HC = a.num_kv_heads * a.n_chunks;
+  const int G = a.heads_per_unit;
 
   const int gid = lane >> 2;  // mma row group
   const int tig = lane & 3;   // thread in group
@@ -96,108 +114,96 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int mi = lane >> 3, mr = lane & 7;
   const int ka_tok = 8 * (mi & 1) + mr, ka_c = mi >> 1;  // K as A (non-transposed)
   const int va_tok = 8 * (mi >> 1) + mr, va_c = mi & 1;  // V^T as A (transposed)
-  const int G = a.heads_per_unit;
+  const int ha = 2 * tig, hb = 2 * tig + 1;              // this lane's head columns
   uint32_t iter = 0;
+  TileProducer prod;
 
-  UnitList list(a, WARPS);
-  int L0 = 0;
-  const long long first = list.next(a, L0);
-  if (first < 0) return;
-  Unit cur = list.describe(a, first, L0);
-  int ent = unit_table_entry(a, cur, lane);
+  for (long long c = (long long)blockIdx.x * WARPS + warp; c < plan.count; c += (long long)gridDim.x * WARPS) {
+    const long long t0 = c * plan.chunk;
+    const int ntile = (int)min(plan.chunk, plan.total - t0);
+    TilePos cp = locate_tile(pt, S, HC, t0);
+    prod.start(cp);
 
-  while (true) {
-    const int n_parts = cur.work ? (cur.L + a.part_tokens - 1) / a.part_tokens : 1;
-    const int ntiles = (cur.tok_end - cur.tok_begin + TILE - 1) / TILE;
-    const bool bad = __any_sync(FULL, cur.work && lane < cur.nblk && (ent < 0 || (long long)ent >= a.num_blocks));
-
-    auto issue = [&](int j, uint32_t it) {
-      const int tok0 = cur.tok_begin + j * TILE;
-      const int phys = __shfl_sync(FULL, ent, tok0 / a.block_size - cur.blk_begin);
+    auto issue_next = [&](uint32_t it) {
+      const int phys = prod.lookup(a, lane);
+      const int st = (int)(it % STAGES);
+      prod.bad_slots = phys >= 0 ? (prod.bad_slots & ~(1u << st)) : (prod.bad_slots | (1u << st));
       if (lane == 0) {
-        const int st = (int)(it % STAGES);
-        const int row0 = (int)(((long long)phys * a.num_kv_heads + cur.h) * a.block_size + (tok0 % a.block_size));
-        unsigned char *dst = ring + st * STAGE_BYTES;
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
+        if (phys >= 0) {
+          const int row0 = (int)prod.first_row(a, phys);
+          unsigned char *dst = ring + st * STAGE_BYTES;
+          mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
 #pragma unroll
-        for (int b = 0; b < BOXES; ++b) {
-          tma_load_2d(dst + b * 2048, &tmap_k, b * 64, row0, &bars[st]);
-          tma_load_2d(dst + TILE_BYTES + b * 2048, &tmap_v, b * 64, row0, &bars[st]);
-        }
-      }
-    };
-    const bool streams = cur.work && !bad;
-    const int npro = streams ? min(ntiles, STAGES) : 0;
-    for (int j = 0; j < npro; ++j) issue(j, iter + j);
-
-    // Q^T as the B operand: b0 = Q[head gid][16ks + 2tig, +1], b1 = the same 8 dims later
-    uint32_t qb[KSTEPS][2];
-    {
-      const bool row_live = streams && gid < G;
-      const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q + (long long)cur.s * a.q_seq_stride +
-                                                                (long long)(cur.hq0 + (row_live ? gid : 0)) * D);
-#pragma unroll
-      for (int ks = 0; ks < KSTEPS; ++ks) {
-        qb[ks][0] = row_live ? __ldg(qrow + 8 * ks + tig) : 0u;
-        qb[ks][1] = row_live ? __ldg(qrow + 8 * ks + 4 + tig) : 0u;
-      }
-    }
-
-    // look up the next unit and its table entries while the copies are in flight
-    int Ln = 0;
-    const long long nslot = list.next(a, Ln);
-    Unit nxt = cur;
-    int ent_n = 0;
-    if (nslot >= 0) {
-      nxt = list.describe(a, nslot, Ln);
-      ent_n = unit_table_entry(a, nxt, lane);
-    }
-
-    if (!streams) {
-      unit_without_tiles(a, cur, bad, lane, D);
-    } else {
-      // per lane: head columns ha = 2*tig and hb = 2*tig + 1
-      float o[KSTEPS][4];
-#pragma unroll
-      for (int mt = 0; mt < KSTEPS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-      float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
-
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = (int)(iter % STAGES);
-        const uint32_t parity = (iter / STAGES) & 1u;
-        const bool arrived = mbar_wait_bounded(&bars[st], parity, a.wait_limit_ns);
-        if (__any_sync(FULL, !arrived)) {
-          if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
-          const int last = min(ntiles, j + STAGES);
-          for (int jj = j; jj < last; ++jj) {
-            const uint32_t it = iter + (jj - j);
-            mbar_wait_bounded(&bars[it % STAGES], (it / STAGES) & 1u, a.wait_limit_ns);
+          for (int bx = 0; bx < BOXES; ++bx) {
+            tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, row0, &bars[st]);
+            tma_load_2d(dst + TILE_BYTES + bx * 2048, &tmap_v, bx * 64, row0, &bars[st]);
           }
-          return;
+        } else {
+          mbar_arrive(&bars[st]);
         }
+      }
+      advance_tile(prod.pos, pt, S, HC);
+    };
+    const int npro = min(ntile, STAGES);
+    for (int k = 0; k < npro; ++k) issue_next(iter + k);
+
+    uint32_t qb[KSTEPS][2];
+    float o[KSTEPS][4];
+    float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+    int L = 0, hq0 = 0, slot = 0;
+    bool full = false, piece_bad = false;
+
+    for (int k = 0; k < ntile; ++k) {
+      if (k == 0 || cp.j == 0) {  // a new piece: segment (cp.s, cp.hc) from tile cp.j on
+        const int len = min(cp.nt - cp.j, ntile - k);
+        full = (cp.j == 0 && len == cp.nt);
+        slot = (k == 0) ? 0 : 1;
+        hq0 = chunk_first_head(a, cp.hc);
+        L = __ldg(a.context_lens + cp.s);
+        piece_bad = false;
+        // Q^T as the B operand: b0 = Q[head gid][16ks + 2tig, +1], b1 = the same 8 dims later
+        const bool row_live = gid < G;
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q + (long long)cp.s * a.q_seq_stride +
+                                                                  (long long)(hq0 + (row_live ? gid : 0)) * D);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          qb[ks][0] = row_live ? __ldg(qrow + 8 * ks + tig) : 0u;
+          qb[ks][1] = row_live ? __ldg(qrow + 8 * ks + 4 + tig) : 0u;
+          o[ks][0] = o[ks][1] = o[ks][2] = o[ks][3] = 0.f;
+        }
+        ma = mb = -INFINITY;
+        la = lb = 0.f;
+      }
+      const int st = (int)(iter % STAGES);
+      if (!wait_slot<STAGES>(bars, iter, min(STAGES, ntile - k), a.wait_limit_ns, lane)) return;
+      const bool tile_bad = (prod.bad_slots >> st) & 1u;  // warp-uniform
+      uint32_t kf[KSTEPS][4], vf[KSTEPS][4];
+      if (!tile_bad) {
         const uint32_t kt = smem_addr(ring + st * STAGE_BYTES);
         const uint32_t vt = kt + TILE_BYTES;
-        uint32_t kf[KSTEPS][4], vf[KSTEPS][4];
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
           ldsm_x4(kf[ks], kt + swizzled(ka_tok, 2 * ks + ka_c));
           ldsm_x4_trans(vf[ks], vt + swizzled(va_tok, 2 * ks + va_c));
         }
-        __syncwarp();
-        if (j + STAGES < ntiles) issue(j + STAGES, iter + STAGES);
-        ++iter;
-        const int nvalid = min(TILE, cur.tok_end - (cur.tok_begin + j * TILE));
+      }
+      __syncwarp();
+      if (k + STAGES < ntile) issue_next(iter + STAGES);
+      ++iter;
+      piece_bad |= tile_bad;
 
+      if (!piece_bad) {
+        const int nvalid = min(TILE, L - cp.j * TILE);
         // S^T = K Q^T: s0 = (token gid, head ha), s1 = (gid, hb), s2 = (gid + 8, ha), s3 = (gid + 8, hb)
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks) MmaOps<E>::mma(s, kf[ks], qb[ks][0], qb[ks][1]);
+        for (int ks = 0; ks < KSTEPS; ++ks) MmaOps<E>::mma(sc, kf[ks], qb[ks][0], qb[ks][1]);
         const bool lo_live = gid < nvalid, hi_live = gid + 8 < nvalid;
-        const float z0 = lo_live ? s[0] * a.scale_log2 : -INFINITY;
-        const float z1 = lo_live ? s[1] * a.scale_log2 : -INFINITY;
-        const float z2 = hi_live ? s[2] * a.scale_log2 : -INFINITY;
-        const float z3 = hi_live ? s[3] * a.scale_log2 : -INFINITY;
+        const float z0 = lo_live ? sc[0] * a.scale_log2 : -INFINITY;
+        const float z1 = lo_live ? sc[1] * a.scale_log2 : -INFINITY;
+        const float z2 = hi_live ? sc[2] * a.scale_log2 : -INFINITY;
+        const float z3 = hi_live ? sc[3] * a.scale_log2 : -INFINITY;
 
         const bool need = z0 > ma + RESCALE_SLACK || z2 > ma + RESCALE_SLACK || z1 > mb + RESCALE_SLACK ||
                           z3 > mb + RESCALE_SLACK;
@@ -209,7 +215,7 @@ __global__ void __launch_bounds__(WARPS * 32)
             cb = fmaxf(cb, __shfl_xor_sync(FULL, cb, off));
           }
           const float na = fmaxf(ma, ca), nb = fmaxf(mb, cb);
-          const float alpha_a = exp2f(ma - na), alpha_b = exp2f(mb - nb);  // 0 on the first tile
+          const float alpha_a = exp2f(ma - na), alpha_b = exp2f(mb - nb);  // 0 on the piece's first tile
 #pragma unroll
           for (int mt = 0; mt < KSTEPS; ++mt) {
             o[mt][0] *= alpha_a;
@@ -253,51 +259,52 @@ __global__ void __launch_bounds__(WARPS * 32)
         }
       }
 
-      // ---- totals per head column (lanes with the same tig), then store
+      if (cp.j + 1 == cp.nt || k + 1 == ntile) {
+        // ---- end of the piece: totals per head column (lanes with the same tig), then store
+        float lta = la, ltb = lb;
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        la += __shfl_xor_sync(FULL, la, off);
-        lb += __shfl_xor_sync(FULL, lb, off);
+        for (int off = 4; off < 32; off <<= 1) {
+          lta += __shfl_xor_sync(FULL, lta, off);
+          ltb += __shfl_xor_sync(FULL, ltb, off);
+        }
+        if (piece_bad && lane == 0) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
+        if (full) {
+          // normalise, narrow, transpose 8x8 blocks back to [head][dims]: lane then holds head gid, dims 2tig, 2tig+1
+          const float ia = piece_bad ? 0.f : 1.f / lta, ib = piece_bad ? 0.f : 1.f / ltb;
+          uint16_t *orow = a.out + (long long)cp.s * a.out_seq_stride + (long long)(hq0 + (gid < G ? gid : 0)) * D + 2 * tig;
+#pragma unroll
+          for (int mt = 0; mt < KSTEPS; ++mt) {
+            const uint32_t t0w = movmatrix_trans(E::narrow2(piece_bad ? 0.f : o[mt][0] * ia, piece_bad ? 0.f : o[mt][1] * ib));
+            const uint32_t t1w = movmatrix_trans(E::narrow2(piece_bad ? 0.f : o[mt][2] * ia, piece_bad ? 0.f : o[mt][3] * ib));
+            if (gid < G) {
+              *reinterpret_cast<uint32_t *>(orow + 16 * mt) = t0w;
+              *reinterpret_cast<uint32_t *>(orow + 16 * mt + 8) = t1w;
+            }
+          }
+        } else {
+          const long long prow = (c * 2 + slot) * G;
+          if (!piece_bad) {
+#pragma unroll
+            for (int mt = 0; mt < KSTEPS; ++mt) {
+              const int d0 = 16 * mt + gid;
+              if (ha < G) {
+                a.ws_acc[(prow + ha) * D + d0] = o[mt][0];
+                a.ws_acc[(prow + ha) * D + d0 + 8] = o[mt][2];
+              }
+              if (hb < G) {
+                a.ws_acc[(prow + hb) * D + d0] = o[mt][1];
+                a.ws_acc[(prow + hb) * D + d0 + 8] = o[mt][3];
+              }
+            }
+          }
+          if (gid == 0) {
+            if (ha < G) a.ws_ml[prow + ha] = piece_bad ? make_float2(-INFINITY, -1.f) : make_float2(ma, lta);
+            if (hb < G) a.ws_ml[prow + hb] = piece_bad ? make_float2(-INFINITY, -1.f) : make_float2(mb, ltb);
+          }
+        }
       }
-      const int ha = 2 * tig, hb = 2 * tig + 1;
-      if (n_parts == 1) {
-        // normalise, narrow, transpose 8x8 blocks back to [head][dims]: lane then holds head gid, dims 2tig, 2tig+1
-        const float ia = 1.f / la, ib = 1.f / lb;
-        uint16_t *orow = a.out + (long long)cur.s * a.out_seq_stride + (long long)(cur.hq0 + gid) * D + 2 * tig;
-#pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt) {
-          const uint32_t t0 = movmatrix_trans(E::narrow2(o[mt][0] * ia, o[mt][1] * ib));
-          const uint32_t t1 = movmatrix_trans(E::narrow2(o[mt][2] * ia, o[mt][3] * ib));
-          if (gid < G) {
-            *reinterpret_cast<uint32_t *>(orow + 16 * mt) = t0;
-            *reinterpret_cast<uint32_t *>(orow + 16 * mt + 8) = t1;
-          }
-        }
-      } else {
-        const long long row_a = ((long long)cur.s * a.num_q_heads + cur.hq0 + ha) * a.n_part_max + cur.p;
-        const long long row_b = row_a + a.n_part_max;
-#pragma unroll
-        for (int mt = 0; mt < KSTEPS; ++mt) {
-          const int d0 = 16 * mt + gid;
-          if (ha < G) {
-            a.ws_acc[row_a * D + d0] = o[mt][0];
-            a.ws_acc[row_a * D + d0 + 8] = o[mt][2];
-          }
-          if (hb < G) {
-            a.ws_acc[row_b * D + d0] = o[mt][1];
-            a.ws_acc[row_b * D + d0 + 8] = o[mt][3];
-          }
-        }
-        if (gid == 0) {
-          if (ha < G) a.ws_ml[row_a] = make_float2(ma, la);
-          if (hb < G) a.ws_ml[row_b] = make_float2(mb, lb);
-        }
-      }
+      advance_tile(cp, pt, S, HC);
     }
-
-    if (nslot < 0) break;
-    cur = nxt;
-    ent = ent_n;
   }
 }
 
