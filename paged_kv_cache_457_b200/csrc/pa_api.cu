@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -78,7 +79,48 @@ int heads_per_unit(int group) {
 #ifndef PA_STAGES
 #define PA_STAGES 2
 #endif
+#ifndef PA_CHUNKS_PER_WARP
+#define PA_CHUNKS_PER_WARP 8
+#endif
+#ifndef PA_MMA_CHUNKS_PER_WARP
+#define PA_MMA_CHUNKS_PER_WARP 1
+#endif
 constexpr int kWarps = PA_WARPS, kStages = PA_STAGES;
+// Balanced split: stream chunks per resident warp.  Measured on B200: the
+// CUDA-core kernel gains from several (fine tail balancing); the tensor-core
+// kernel, whose cut pieces carry up to 8 heads each to merge, prefers one.
+constexpr int kChunksPerWarp = PA_CHUNKS_PER_WARP;
+constexpr int kMmaChunksPerWarp = PA_MMA_CHUNKS_PER_WARP;
+int chunks_per_warp(int group) { return uses_mma(group) ? kMmaChunksPerWarp : kChunksPerWarp; }
+
+// Launches `kernel` with programmatic stream serialisation allowed: it may start
+// while the previous kernel in the stream finishes, and waits for it on the
+// device (griddepcontrol.wait) before touching any input.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Per-call tag of the chunk counter (never 0: the merge kernel leaves the counter at 0).
+std::atomic<uint32_t> g_epoch{0x9e3779b9u};
+uint32_t next_epoch() {
+  uint32_t e;
+  do {
+    e = g_epoch.fetch_add(0x61c88647u, std::memory_order_relaxed);
+  } while (e == 0);
+  return e;
+}
 constexpr int kMaxSeqs = 32768;         // tile prefix kept in shared memory
 
 template <class E, int D>
@@ -157,7 +199,7 @@ struct LaunchPlan {
   int grid;          // blocks of the split kernel (for `dtype`; 0 if not asked)
   long long max_chunks;
   int chunk_tiles;   // 0: balanced
-  size_t tiles_bytes, ml_bytes, acc_bytes, total_bytes;
+  size_t queue_bytes, tiles_bytes, ml_bytes, acc_bytes, total_bytes;
 };
 
 int plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
@@ -177,16 +219,17 @@ int plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, i
   lp->grid = dtype == 0 ? 0 : sms * (dtype == PA_BFLOAT16 ? occ_bf16 : occ_f16);
   lp->chunk_tiles = partition_tokens / pa::TILE;
   if (lp->chunk_tiles == 0) {
-    lp->max_chunks = ws_warps;
+    lp->max_chunks = ws_warps * chunks_per_warp(group);
   } else {
     const long long per_seq = ((long long)max_context_len + pa::TILE - 1) / pa::TILE;
     const long long total = (long long)num_seqs * num_kv_heads * (group / G) * per_seq;
     lp->max_chunks = std::max(1LL, (total + lp->chunk_tiles - 1) / lp->chunk_tiles);
   }
+  lp->queue_bytes = 256;
   lp->tiles_bytes = (((size_t)num_seqs + 1) * sizeof(int) + 255) / 256 * 256;
   lp->ml_bytes = (size_t)lp->max_chunks * 2 * G * sizeof(float2);
   lp->acc_bytes = (size_t)lp->max_chunks * 2 * G * head_dim * sizeof(float);
-  lp->total_bytes = lp->tiles_bytes + lp->ml_bytes + lp->acc_bytes;
+  lp->total_bytes = lp->queue_bytes + lp->tiles_bytes + lp->ml_bytes + lp->acc_bytes;
   return PA_OK;
 }
 
@@ -271,18 +314,25 @@ int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype,
     if (rc != PA_OK) return rc;
     rc = cache_tensor_map(args.v_cache, rows, D, dtype, &mv);
     if (rc != PA_OK) return rc;
-    pa::decode_split_mma_kernel<E, D, kWarps, kStages><<<lp.grid, threads, lp.smem, stream>>>(mk, mv, args);
+    cudaError_t e = launch_pdl(pa::decode_split_mma_kernel<E, D, kWarps, kStages>, dim3(lp.grid), dim3(threads),
+                               lp.smem, stream, mk, mv, args);
+    if (e != cudaSuccess) return record(e);
   } else if (args.heads_per_unit == 2) {
-    pa::decode_split_kernel<E, D, 2, kWarps, kStages><<<lp.grid, threads, lp.smem, stream>>>(args);
+    cudaError_t e = launch_pdl(pa::decode_split_kernel<E, D, 2, kWarps, kStages>, dim3(lp.grid), dim3(threads),
+                               lp.smem, stream, args);
+    if (e != cudaSuccess) return record(e);
   } else {
-    pa::decode_split_kernel<E, D, 1, kWarps, kStages><<<lp.grid, threads, lp.smem, stream>>>(args);
+    cudaError_t e = launch_pdl(pa::decode_split_kernel<E, D, 1, kWarps, kStages>, dim3(lp.grid), dim3(threads),
+                               lp.smem, stream, args);
+    if (e != cudaSuccess) return record(e);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   const long long warps = (long long)args.num_seqs * args.num_q_heads;
   const int grid = (int)std::max(1LL, std::min<long long>((warps + 7) / 8, (long long)sms * 8));
-  pa::decode_merge_kernel<E, D><<<grid, 256, 0, stream>>>(args);
+  e = launch_pdl(pa::decode_merge_kernel<E, D>, dim3(grid), dim3(256), 0, stream, args);
+  if (e != cudaSuccess) return record(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -352,8 +402,9 @@ int pa_write_kv(const void *k, const void *v, void *k_cache, void *v_cache, cons
   a.block_size = block_size;
   const long long chunks = 2LL * num_tokens * num_kv_heads * (head_dim / 8);
   const int grid = (int)std::max(1LL, std::min<long long>((chunks + 255) / 256, (long long)sms * 8));
-  pa::write_kv_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(pa::write_kv_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), a);
+  if (e != cudaSuccess) return record(e);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return PA_OK;
@@ -405,9 +456,10 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.out = static_cast<uint16_t *>(out);
-  a.ws_tiles = reinterpret_cast<int *>(ws);
-  a.ws_ml = reinterpret_cast<float2 *>(ws + lp.tiles_bytes);
-  a.ws_acc = reinterpret_cast<float *>(ws + lp.tiles_bytes + lp.ml_bytes);
+  a.ws_queue = reinterpret_cast<unsigned long long *>(ws);
+  a.ws_tiles = reinterpret_cast<int *>(ws + lp.queue_bytes);
+  a.ws_ml = reinterpret_cast<float2 *>(ws + lp.queue_bytes + lp.tiles_bytes);
+  a.ws_acc = reinterpret_cast<float *>(ws + lp.queue_bytes + lp.tiles_bytes + lp.ml_bytes);
   a.num_blocks = num_blocks;
   a.q_seq_stride = q_seq_stride;
   a.out_seq_stride = out_seq_stride;
@@ -425,6 +477,8 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   a.n_chunks = group / G;
   a.chunk_tiles = lp.chunk_tiles;
   a.split_warps = lp.grid * kWarps;
+  a.chunks_per_warp = chunks_per_warp(group);
+  a.epoch = next_epoch();
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == PA_BFLOAT16;

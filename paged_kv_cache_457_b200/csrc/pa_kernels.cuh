@@ -90,6 +90,8 @@ struct WriteArgs {
 
 // One thread per 16-byte chunk of a (token, kv head) row, K rows then V rows.
 __global__ void __launch_bounds__(256) write_kv_kernel(const WriteArgs a) {
+  grid_dependency_wait();  // the new rows may come from the previous kernel in the stream
+  grid_launch_dependents();
   const int cpr = a.head_dim / 8;
   const long long per = a.num_tokens * a.num_kv_heads * cpr;
   const long long cap = a.num_blocks * a.block_size;
@@ -135,6 +137,7 @@ struct DecodeArgs {
   const int32_t *block_tables;
   const int32_t *context_lens;
   uint16_t *out;
+  unsigned long long *ws_queue;  // chunk queue word: (call epoch << 32) | next ticket; reset to 0 by the merge kernel
   int *ws_tiles;   // [num_seqs + 1] tile prefix, written by block 0 of the split kernel for the merge kernel
   float2 *ws_ml;   // [max_chunks][2][heads_per_unit] (running max in base-2 units, running sum) of partial pieces
   float *ws_acc;   // [max_chunks][2][heads_per_unit][head_dim] un-normalised partial outputs
@@ -147,6 +150,8 @@ struct DecodeArgs {
   int heads_per_unit;  // query heads per head chunk (group / n_chunks)
   int chunk_tiles;     // tiles per chunk; 0: total tiles / split_warps
   int split_warps;     // warps in the split kernel's grid
+  int chunks_per_warp; // balanced split: target chunks per warp (the first one static, the rest from the queue)
+  unsigned epoch;      // non-zero, different for every call
 };
 
 __device__ __forceinline__ bool context_ok(const DecodeArgs &a, int L) {
@@ -190,23 +195,63 @@ __device__ __forceinline__ void build_tile_prefix(const DecodeArgs &a, int *pt, 
   __syncthreads();
 }
 
-constexpr int MIN_AUTO_CHUNK_TILES = 4;  // the balanced split never cuts finer than this
+constexpr int MIN_CHUNK_TILES = 4;  // never cut the stream finer than this (>= ring depth)
 
 struct ChunkPlan {
   long long total, chunk, count;
+  __device__ __forceinline__ int length(long long c) const { return (int)min(chunk, total - c * chunk); }
 };
 
-// Chunk length and count for a tile stream of pt[S] * head_chunks tiles.
-__device__ __forceinline__ ChunkPlan plan_chunks(const DecodeArgs &a, int tiles_per_chunk_set) {
+// Chunk length and count for a tile stream of tiles_per_head_chunk_set * head_chunks tiles.
+__device__ __forceinline__ ChunkPlan plan_chunks(const DecodeArgs &a, int tiles_per_head_chunk_set) {
   ChunkPlan p;
-  p.total = (long long)tiles_per_chunk_set * a.num_kv_heads * a.n_chunks;
-  long long c = a.chunk_tiles > 0 ? a.chunk_tiles
-                                  : max((p.total + a.split_warps - 1) / a.split_warps, (long long)MIN_AUTO_CHUNK_TILES);
+  p.total = (long long)tiles_per_head_chunk_set * a.num_kv_heads * a.n_chunks;
+  const long long target = (long long)a.split_warps * a.chunks_per_warp;
+  long long c = a.chunk_tiles > 0 ? a.chunk_tiles : (p.total + target - 1) / target;
   c = max(c, (p.total + a.max_chunks - 1) / a.max_chunks);  // never more chunks than the workspace holds
-  p.chunk = max(c, 1LL);
+  p.chunk = max(c, (long long)MIN_CHUNK_TILES);
   p.count = (p.total + p.chunk - 1) / p.chunk;
   return p;
 }
+
+// Chunk hand-out: chunk w goes to warp w; later chunks come from a counter in
+// the workspace.  Block 0 installs (epoch << 32) in the counter word at the
+// start of the call (the epoch is non-zero and new for every call, and the
+// merge kernel leaves the word at 0), so a ticket drawn before the install is
+// recognised by its stale upper half and drawn again.  Tickets are requested
+// half a chunk ahead of need.
+struct ChunkQueue {
+  unsigned long long *word;
+  unsigned epoch;
+  long long first_dynamic, count;
+  unsigned long long pending;  // lane 0: result of the last atomicAdd
+
+  __device__ __forceinline__ void request(int lane) {
+    if (lane == 0) pending = atomicAdd(word, 1ull);
+  }
+  // The chunk of the last request (>= count: none left).
+  __device__ __forceinline__ long long take(int lane, unsigned long long limit_ns) {
+    unsigned long long ticket = 0;
+    if (lane == 0) {
+      unsigned long long old = pending;
+      const uint64_t t0 = global_ns();
+      while ((unsigned)(old >> 32) != epoch) {  // drawn before this call's counter was installed
+        if (global_ns() - t0 > limit_ns) {
+          atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
+          old = ~0ull;
+          break;
+        }
+        __nanosleep(256);
+        old = atomicAdd(word, 1ull);
+      }
+      ticket = old == ~0ull ? ~0ull : (old & 0xffffffffull);
+    }
+    ticket = __shfl_sync(FULL, ticket, 0);
+    if (ticket == ~0ull) return count;
+    const long long c = first_dynamic + (long long)ticket;
+    return c < count ? c : count;
+  }
+};
 
 // A position in the tile stream: tile j of head chunk hc of sequence s (nt tiles).
 struct TilePos {
@@ -381,7 +426,7 @@ __device__ __forceinline__ bool wait_slot(uint64_t *bars, uint32_t it, int in_fl
 constexpr float RESCALE_SLACK = 8.f;
 
 template <class E, int D, int G, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(const DecodeArgs a) {
   constexpr int LPR = D / 8;       // lanes covering one K/V row
   constexpr int NGRP = 32 / LPR;   // rows one warp-wide 16-byte load covers
   constexpr int R = TILE / NGRP;   // rows per lane per tile
@@ -400,6 +445,9 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
     for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
   }
+  grid_dependency_wait();    // every input may come from the previous kernel in the stream
+  grid_launch_dependents();  // the merge kernel may launch now and wait for this grid
+  if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(a.ws_queue, (unsigned long long)a.epoch << 32);
   const int S = a.num_seqs;
   build_tile_prefix(a, pt, pt + S + 1);
   if (blockIdx.x == 0)
@@ -413,13 +461,33 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
   uint32_t iter = 0;  // tiles consumed by this warp: ring slot iter % STAGES, phase (iter / STAGES) & 1
   TileProducer prod;
 
-  for (long long c = (long long)blockIdx.x * WARPS + warp; c < plan.count; c += (long long)gridDim.x * WARPS) {
-    const long long t0 = c * plan.chunk;
-    const int ntile = (int)min(plan.chunk, plan.total - t0);
-    TilePos cp = locate_tile(pt, S, HC, t0);
+  long long cons_c = (long long)blockIdx.x * WARPS + warp;  // chunk the consumer is in (the first one is static)
+  if (cons_c < plan.count) {
+    ChunkQueue queue{a.ws_queue, a.epoch, (long long)a.split_warps, plan.count, 0ull};
+    bool requested = false;  // a ticket for the producer's next chunk is on its way
+    long long prod_c = cons_c;
+    int prod_left = plan.length(prod_c);
+    bool prod_done = false;
+    TilePos cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
     prod.start(cp);
+    uint32_t issued = iter;  // tiles issued by this warp: the next goes to ring slot issued % STAGES
 
-    auto issue_next = [&](uint32_t it) {
+    // issue the producer's next tile, moving it into its next chunk when the current one is done
+    auto issue_next = [&]() {
+      if (prod_left == 0) {
+        if (prod_done) return;
+        if (!requested) queue.request(lane);
+        requested = false;
+        const long long nc = queue.take(lane, a.wait_limit_ns);
+        if (nc >= plan.count) {
+          prod_done = true;
+          return;
+        }
+        prod_c = nc;
+        prod_left = plan.length(nc);
+        prod.start(locate_tile(pt, S, HC, nc * plan.chunk));
+      }
+      const uint32_t it = issued++;
       const int phys = prod.lookup(a, lane);
       const int st = (int)(it % STAGES);
       prod.bad_slots = phys >= 0 ? (prod.bad_slots & ~(1u << st)) : (prod.bad_slots | (1u << st));
@@ -436,9 +504,13 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
         }
       }
       advance_tile(prod.pos, pt, S, HC);
+      --prod_left;
+      if (!requested && 2 * prod_left <= plan.length(prod_c)) {
+        queue.request(lane);
+        requested = true;
+      }
     };
-    const int npro = min(ntile, STAGES);
-    for (int k = 0; k < npro; ++k) issue_next(iter + k);
+    for (int k = 0; k < STAGES; ++k) issue_next();
 
     uint32_t qw[G][4];
     float m[G], lsum[G];
@@ -446,9 +518,18 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
     int L = 0, hq0 = 0, slot = 0;
     bool full = false, piece_bad = false;
 
-    for (int k = 0; k < ntile; ++k) {
+    int cons_left = plan.length(cons_c);
+    int k = 0;  // tile index within the consumer's chunk
+    while (true) {
+      if (cons_left == 0) {  // the consumer's chunk is done: follow the producer into its next chunk
+        if (prod_c == cons_c) break;
+        cons_c = prod_c;
+        cons_left = plan.length(cons_c);
+        cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
+        k = 0;
+      }
       if (k == 0 || cp.j == 0) {  // a new piece: segment (cp.s, cp.hc) from tile cp.j on
-        const int len = min(cp.nt - cp.j, ntile - k);
+        const int len = min(cp.nt - cp.j, cons_left);
         full = (cp.j == 0 && len == cp.nt);
         slot = (k == 0) ? 0 : 1;
         hq0 = chunk_first_head(a, cp.hc);
@@ -469,7 +550,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
         }
       }
       const int st = (int)(iter % STAGES);
-      if (!wait_slot<STAGES>(bars, iter, min(STAGES, ntile - k), a.wait_limit_ns, lane)) return;
+      if (!wait_slot<STAGES>(bars, iter, (int)(issued - iter), a.wait_limit_ns, lane)) return;
       const bool tile_bad = (prod.bad_slots >> st) & 1u;
       // copy this lane's rows out of the slot, then hand the slot straight back to the copy engine
       const unsigned char *kt = ring + st * STAGE_BYTES;
@@ -483,7 +564,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
                          : *reinterpret_cast<const uint4 *>(vt + ((r * NGRP + grp) * D + cl * 8) * 2);
       }
       __syncwarp();
-      if (k + STAGES < ntile) issue_next(iter + STAGES);
+      issue_next();
       ++iter;
       piece_bad |= tile_bad;
 
@@ -541,7 +622,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
         }
       }
 
-      if (cp.j + 1 == cp.nt || k + 1 == ntile) {
+      if (cp.j + 1 == cp.nt || cons_left == 1) {
         // ---- end of the piece: merge the row groups, total the sums, store the output or the partial
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
@@ -574,7 +655,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
             }
           }
         } else {
-          const long long prow = (c * 2 + slot) * G;
+          const long long prow = (cons_c * 2 + slot) * G;
 #pragma unroll
           for (int gg = 0; gg < G; ++gg) {
             if (lane < LPR && !piece_bad) {
@@ -587,6 +668,8 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const DecodeAr
         }
       }
       advance_tile(cp, pt, S, HC);
+      --cons_left;
+      ++k;
     }
   }
 }
@@ -600,6 +683,9 @@ template <class E, int D>
 __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
   constexpr int DPL = D / 32;  // dims per lane (4 or 2)
   const int lane = threadIdx.x & 31;
+  grid_dependency_wait();  // the split kernel's pieces and tile prefix
+  grid_launch_dependents();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ws_queue = 0ull;  // leave the chunk counter clear
   const int S = a.num_seqs;
   const ChunkPlan plan = plan_chunks(a, a.ws_tiles[S]);
   const int HC = a.num_kv_heads * a.n_chunks;

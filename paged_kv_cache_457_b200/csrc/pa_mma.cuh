@@ -76,7 +76,7 @@ struct MmaSmem {
 };
 
 template <class E, int D, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32)
+__global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
     decode_split_mma_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                             const DecodeArgs a) {
   constexpr int KSTEPS = D / 16;  // 16-dim steps of QK^T, and 16-dim row tiles of O^T
@@ -100,6 +100,9 @@ __global__ void __launch_bounds__(WARPS * 32)
     prefetch_tensor_map(&tmap_k);
     prefetch_tensor_map(&tmap_v);
   }
+  grid_dependency_wait();    // every input may come from the previous kernel in the stream
+  grid_launch_dependents();  // the merge kernel may launch now and wait for this grid
+  if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(a.ws_queue, (unsigned long long)a.epoch << 32);
   const int S = a.num_seqs;
   build_tile_prefix(a, pt, pt + S + 1);
   if (blockIdx.x == 0)
@@ -118,13 +121,33 @@ __global__ void __launch_bounds__(WARPS * 32)
   uint32_t iter = 0;
   TileProducer prod;
 
-  for (long long c = (long long)blockIdx.x * WARPS + warp; c < plan.count; c += (long long)gridDim.x * WARPS) {
-    const long long t0 = c * plan.chunk;
-    const int ntile = (int)min(plan.chunk, plan.total - t0);
-    TilePos cp = locate_tile(pt, S, HC, t0);
+  long long cons_c = (long long)blockIdx.x * WARPS + warp;  // chunk the consumer is in (the first one is static)
+  if (cons_c < plan.count) {
+    ChunkQueue queue{a.ws_queue, a.epoch, (long long)a.split_warps, plan.count, 0ull};
+    bool requested = false;  // a ticket for the producer's next chunk is on its way
+    long long prod_c = cons_c;
+    int prod_left = plan.length(prod_c);
+    bool prod_done = false;
+    TilePos cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
     prod.start(cp);
+    uint32_t issued = iter;  // tiles issued by this warp: the next goes to ring slot issued % STAGES
 
-    auto issue_next = [&](uint32_t it) {
+    // issue the producer's next tile, moving it into its next chunk when the current one is done
+    auto issue_next = [&]() {
+      if (prod_left == 0) {
+        if (prod_done) return;
+        if (!requested) queue.request(lane);
+        requested = false;
+        const long long nc = queue.take(lane, a.wait_limit_ns);
+        if (nc >= plan.count) {
+          prod_done = true;
+          return;
+        }
+        prod_c = nc;
+        prod_left = plan.length(nc);
+        prod.start(locate_tile(pt, S, HC, nc * plan.chunk));
+      }
+      const uint32_t it = issued++;
       const int phys = prod.lookup(a, lane);
       const int st = (int)(it % STAGES);
       prod.bad_slots = phys >= 0 ? (prod.bad_slots & ~(1u << st)) : (prod.bad_slots | (1u << st));
@@ -144,9 +167,13 @@ __global__ void __launch_bounds__(WARPS * 32)
         }
       }
       advance_tile(prod.pos, pt, S, HC);
+      --prod_left;
+      if (!requested && 2 * prod_left <= plan.length(prod_c)) {
+        queue.request(lane);
+        requested = true;
+      }
     };
-    const int npro = min(ntile, STAGES);
-    for (int k = 0; k < npro; ++k) issue_next(iter + k);
+    for (int k = 0; k < STAGES; ++k) issue_next();
 
     uint32_t qb[KSTEPS][2];
     float o[KSTEPS][4];
@@ -154,9 +181,18 @@ __global__ void __launch_bounds__(WARPS * 32)
     int L = 0, hq0 = 0, slot = 0;
     bool full = false, piece_bad = false;
 
-    for (int k = 0; k < ntile; ++k) {
+    int cons_left = plan.length(cons_c);
+    int k = 0;  // tile index within the consumer's chunk
+    while (true) {
+      if (cons_left == 0) {  // the consumer's chunk is done: follow the producer into its next chunk
+        if (prod_c == cons_c) break;
+        cons_c = prod_c;
+        cons_left = plan.length(cons_c);
+        cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
+        k = 0;
+      }
       if (k == 0 || cp.j == 0) {  // a new piece: segment (cp.s, cp.hc) from tile cp.j on
-        const int len = min(cp.nt - cp.j, ntile - k);
+        const int len = min(cp.nt - cp.j, cons_left);
         full = (cp.j == 0 && len == cp.nt);
         slot = (k == 0) ? 0 : 1;
         hq0 = chunk_first_head(a, cp.hc);
@@ -176,29 +212,31 @@ __global__ void __launch_bounds__(WARPS * 32)
         la = lb = 0.f;
       }
       const int st = (int)(iter % STAGES);
-      if (!wait_slot<STAGES>(bars, iter, min(STAGES, ntile - k), a.wait_limit_ns, lane)) return;
+      if (!wait_slot<STAGES>(bars, iter, (int)(issued - iter), a.wait_limit_ns, lane)) return;
       const bool tile_bad = (prod.bad_slots >> st) & 1u;  // warp-uniform
-      uint32_t kf[KSTEPS][4], vf[KSTEPS][4];
-      if (!tile_bad) {
+      piece_bad |= tile_bad;
+      // S^T = K Q^T (K fragments loaded just before use), then the V^T fragments; then the slot is free
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t vf[KSTEPS][4];
+      if (!piece_bad) {
         const uint32_t kt = smem_addr(ring + st * STAGE_BYTES);
         const uint32_t vt = kt + TILE_BYTES;
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
-          ldsm_x4(kf[ks], kt + swizzled(ka_tok, 2 * ks + ka_c));
-          ldsm_x4_trans(vf[ks], vt + swizzled(va_tok, 2 * ks + va_c));
+          uint32_t kf[4];
+          ldsm_x4(kf, kt + swizzled(ka_tok, 2 * ks + ka_c));
+          MmaOps<E>::mma(sc, kf, qb[ks][0], qb[ks][1]);
         }
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) ldsm_x4_trans(vf[ks], vt + swizzled(va_tok, 2 * ks + va_c));
       }
       __syncwarp();
-      if (k + STAGES < ntile) issue_next(iter + STAGES);
+      issue_next();
       ++iter;
-      piece_bad |= tile_bad;
 
       if (!piece_bad) {
         const int nvalid = min(TILE, L - cp.j * TILE);
-        // S^T = K Q^T: s0 = (token gid, head ha), s1 = (gid, hb), s2 = (gid + 8, ha), s3 = (gid + 8, hb)
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks) MmaOps<E>::mma(sc, kf[ks], qb[ks][0], qb[ks][1]);
+        // s0 = (token gid, head ha), s1 = (gid, hb), s2 = (gid + 8, ha), s3 = (gid + 8, hb)
         const bool lo_live = gid < nvalid, hi_live = gid + 8 < nvalid;
         const float z0 = lo_live ? sc[0] * a.scale_log2 : -INFINITY;
         const float z1 = lo_live ? sc[1] * a.scale_log2 : -INFINITY;
@@ -259,7 +297,7 @@ __global__ void __launch_bounds__(WARPS * 32)
         }
       }
 
-      if (cp.j + 1 == cp.nt || k + 1 == ntile) {
+      if (cp.j + 1 == cp.nt || cons_left == 1) {
         // ---- end of the piece: totals per head column (lanes with the same tig), then store
         float lta = la, ltb = lb;
 #pragma unroll
@@ -282,7 +320,7 @@ __global__ void __launch_bounds__(WARPS * 32)
             }
           }
         } else {
-          const long long prow = (c * 2 + slot) * G;
+          const long long prow = (cons_c * 2 + slot) * G;
           if (!piece_bad) {
 #pragma unroll
             for (int mt = 0; mt < KSTEPS; ++mt) {
@@ -304,6 +342,8 @@ __global__ void __launch_bounds__(WARPS * 32)
         }
       }
       advance_tile(cp, pt, S, HC);
+      --cons_left;
+      ++k;
     }
   }
 }
