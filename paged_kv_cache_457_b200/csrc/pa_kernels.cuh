@@ -677,8 +677,9 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
 // One warp per (sequence, query head): writes the zero rows of empty or
 // invalid sequences (setting the status bits of the invalid ones) and merges
 // the partial pieces of segments that the split kernel cut across chunks:
-// out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p, M = max_p m_p, in
-// increasing chunk order (deterministic).
+// out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p, M = max_p m_p, summed
+// in increasing chunk order (deterministic).  Built for latency: lane p holds
+// piece p's (m, l) and weight, and the partial rows are loaded eight at a time.
 template <class E, int D>
 __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
   constexpr int DPL = D / 32;  // dims per lane (4 or 2)
@@ -687,14 +688,16 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
   grid_launch_dependents();
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.ws_queue = 0ull;  // leave the chunk counter clear
   const int S = a.num_seqs;
-  const ChunkPlan plan = plan_chunks(a, a.ws_tiles[S]);
+  const ChunkPlan plan = plan_chunks(a, __ldg(a.ws_tiles + S));
   const int HC = a.num_kv_heads * a.n_chunks;
+  const int G = a.heads_per_unit;
   const long long total = (long long)S * a.num_q_heads;
   const long long nw = (long long)gridDim.x * (blockDim.x / 32);
   for (long long w = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); w < total; w += nw) {
     const int s = (int)(w / a.num_q_heads);
     const int hq = (int)(w - (long long)s * a.num_q_heads);
     const int L = __ldg(a.context_lens + s);
+    const int pt0 = __ldg(a.ws_tiles + s), pt1 = __ldg(a.ws_tiles + s + 1);
     uint16_t *dst = a.out + (long long)s * a.out_seq_stride + (long long)hq * D + lane * DPL;
     float o[DPL];
 #pragma unroll
@@ -707,17 +710,25 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
     } else {
       const int h = hq / a.group;
       const int r = hq - h * a.group;
-      const int ch = r / a.heads_per_unit;
-      const int gg = r - ch * a.heads_per_unit;
-      const int nt = a.ws_tiles[s + 1] - a.ws_tiles[s];
-      const long long seg0 = (long long)a.ws_tiles[s] * HC + (long long)(h * a.n_chunks + ch) * nt;
+      const int ch = r / G;
+      const int gg = r - ch * G;
+      const int nt = pt1 - pt0;
+      const long long seg0 = (long long)pt0 * HC + (long long)(h * a.n_chunks + ch) * nt;
       const long long c_first = seg0 / plan.chunk, c_last = (seg0 + nt - 1) / plan.chunk;
       if (c_first == c_last) continue;  // one chunk held the whole segment: the split kernel wrote the row
-      float M = -INFINITY;
-      bool err = false;
-      for (long long c = c_first + lane; c <= c_last; c += 32) {
-        const int slot = (c == c_first && seg0 > c * plan.chunk) ? 1 : 0;
-        const float2 ml = a.ws_ml[(c * 2 + slot) * a.heads_per_unit + gg];
+      const int n = (int)(c_last - c_first + 1);
+      auto piece_row = [&](int p) -> int {  // partial row of piece p (chunk c_first + p)
+        const long long c = c_first + p;
+        const int slot = (p == 0 && seg0 > c * plan.chunk) ? 1 : 0;
+        return (int)((c * 2 + slot) * G + gg);
+      };
+      // pass 1: maximum and validity over all pieces; lane p keeps piece p of the first 32
+      float2 ml0 = make_float2(-INFINITY, 0.f);
+      if (lane < n) ml0 = __ldg(a.ws_ml + piece_row(lane));
+      float M = ml0.x;
+      bool err = lane < n && ml0.y < 0.f;
+      for (int p = lane + 32; p < n; p += 32) {
+        const float2 ml = __ldg(a.ws_ml + piece_row(p));
         M = fmaxf(M, ml.x);
         err |= ml.y < 0.f;
       }
@@ -726,24 +737,33 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
       err = __any_sync(FULL, err);
       if (!err) {
         float l = 0.f;
-        for (long long c = c_first; c <= c_last; ++c) {
-          const int slot = (c == c_first && seg0 > c * plan.chunk) ? 1 : 0;
-          const long long row = (c * 2 + slot) * a.heads_per_unit + gg;
-          const float2 ml = a.ws_ml[row];
-          const float wgt = exp2f(ml.x - M);
+        for (int base = 0; base < n; base += 32) {
+          const int p = base + lane;
+          const float2 ml = base == 0 ? ml0 : (p < n ? __ldg(a.ws_ml + piece_row(p)) : make_float2(-INFINITY, 0.f));
+          const float wgt = p < n ? exp2f(ml.x - M) : 0.f;
+          const int row = p < n ? piece_row(p) : 0;
           l = fmaf(ml.y, wgt, l);
-          const float *src = a.ws_acc + row * D + lane * DPL;
-          float v[DPL];
-          if constexpr (DPL == 4) {
-            const float4 t = *reinterpret_cast<const float4 *>(src);
-            v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-          } else {
-            const float2 t = *reinterpret_cast<const float2 *>(src);
-            v[0] = t.x; v[1] = t.y;
+          const int cnt = min(32, n - base);
+#pragma unroll 8
+          for (int q = 0; q < cnt; ++q) {
+            const float wq = __shfl_sync(FULL, wgt, q);
+            const int rq = __shfl_sync(FULL, row, q);
+            const float *src = a.ws_acc + (long long)rq * D + lane * DPL;
+            if constexpr (DPL == 4) {
+              const float4 t = __ldg(reinterpret_cast<const float4 *>(src));
+              o[0] = fmaf(wq, t.x, o[0]);
+              o[1] = fmaf(wq, t.y, o[1]);
+              o[2] = fmaf(wq, t.z, o[2]);
+              o[3] = fmaf(wq, t.w, o[3]);
+            } else {
+              const float2 t = __ldg(reinterpret_cast<const float2 *>(src));
+              o[0] = fmaf(wq, t.x, o[0]);
+              o[1] = fmaf(wq, t.y, o[1]);
+            }
           }
-#pragma unroll
-          for (int k = 0; k < DPL; ++k) o[k] = fmaf(wgt, v[k], o[k]);
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(FULL, l, off);
 #pragma unroll
         for (int k = 0; k < DPL; ++k) o[k] = o[k] / l;
       }
