@@ -76,6 +76,27 @@ def step_bytes(wl, st):
     return kv, kv + qo + 4 * nblk + 4 * st.num_seqs
 
 
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or (None, reason)
+    when the kernel sources changed since the capture or the workload was not captured."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for rel in rec["kernel_sources"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["kernel_sources_sha256"]:
+            return None, "kernel changed since the ncu capture"
+        w = rec["workloads"].get(workload)
+        if w is None:
+            return None, "no ncu capture for this workload"
+        return int(w["dram_bytes_per_launch"]), w["kernel"] + ": " + w["how"]
+    except (OSError, KeyError, ValueError) as e:
+        return None, f"no traffic record ({type(e).__name__})"
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -357,6 +378,7 @@ def main():
         value = world * kv_b / (ms_step / 1e3) / 1e9
         peak, peak_kind = measured_peak()
         achieved = alg_b / (dec_ms / 1e3) / 1e9
+        traffic, traffic_note = recorded_traffic(wl.name)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -372,7 +394,7 @@ def main():
                        "l2": f"no flush: {kv_b / 1e9:.2f} GB of K/V per step, larger than the 126 MB L2"},
             "roofline": {"bound": "hbm", "kernel": "pa_decode (split + merge kernels)",
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_note": traffic_note,
                          "algorithmic_bytes": alg_b, "ms_per_launch": round(dec_ms, 5)},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": sampler.summary(wall0, wall1), "device_status": status,
