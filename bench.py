@@ -97,6 +97,22 @@ def recorded_traffic(workload: str):
         return None, f"no traffic record ({type(e).__name__})"
 
 
+def max_over_ranks(values, device=None):
+    """Elementwise maximum of per-rank timings (ms) over all ranks; identity on one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_rate_gbs(bytes_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank moves bytes_per_rank_step per step; time = slowest rank."""
+    return world * bytes_per_rank_step * steps / (max_ms / 1e3) / 1e9
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -353,19 +369,12 @@ def main():
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": round(world * kv_b * args.steps / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], device)[0]
+        e2e = {"value": round(job_rate_gbs(kv_b, world, args.steps, e2e_ms), 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e2e_ms / args.steps, 4)}
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms, dec_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, dec_ms = float(t[0].item()), float(t[1].item())
+    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -375,7 +384,7 @@ def main():
 
     if rank == 0:
         ms_step = elapsed_ms / args.steps
-        value = world * kv_b / (ms_step / 1e3) / 1e9
+        value = job_rate_gbs(kv_b, world, args.steps, elapsed_ms)
         peak, peak_kind = measured_peak()
         achieved = alg_b / (dec_ms / 1e3) / 1e9
         traffic, traffic_note = recorded_traffic(wl.name)

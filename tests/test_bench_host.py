@@ -1,0 +1,86 @@
+"""bench.py's host-side logic on the CPU: byte accounting, the traffic record, the max-over-ranks
+timing across two gloo ranks, and the reference arm's JSON line."""
+import json
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+import workloads as W
+
+
+def test_step_bytes_counts_live_tokens_q_out_table_and_lengths():
+    wl = W.custom(seed=1, num_seqs=3, num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16, lens=[1, 16, 40])
+    st = wl.steps[0]
+    kv, alg = bench.step_bytes(wl, st)
+    assert kv == (1 + 16 + 40) * 2 * 64 * 2 * 2
+    assert alg == kv + 2 * 3 * 4 * 64 * 2 + 4 * (1 + 1 + 3) + 4 * 3
+
+
+def test_job_rate_is_whole_job_over_slowest_rank():
+    # 2 ranks x 1 GB per step x 10 steps in 20 ms (the slower rank) = 1000 GB/s
+    assert bench.job_rate_gbs(10**9, 2, 10, 20.0) == pytest.approx(1000.0)
+
+
+def test_traffic_record_requires_matching_kernel_sources(tmp_path, monkeypatch):
+    val, note = bench.recorded_traffic("llama2_7b_decode")
+    assert val is None or val > 0
+    fake = tmp_path / "profiles"
+    fake.mkdir()
+    (tmp_path / "k.cuh").write_text("kernel v1")
+    import hashlib
+    rec = {"kernel_sources": ["k.cuh"], "kernel_sources_sha256": hashlib.sha256(b"kernel v1").hexdigest(),
+           "workloads": {"w": {"kernel": "k", "dram_bytes_per_launch": 123, "how": "test"}}}
+    (fake / "decode_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("w")[0] == 123
+    assert bench.recorded_traffic("other")[0] is None
+    (tmp_path / "k.cuh").write_text("kernel v2")
+    assert bench.recorded_traffic("w") == (None, "kernel changed since the ncu capture")
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local = [10.0 + rank, 5.0 - rank]  # rank 1 is slower on the first figure, faster on the second
+        out[rank] = bench.max_over_ranks(local)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == [11.0, 5.0] and out[1] == [11.0, 5.0]
+
+
+def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "tiny_decode",
+                                      "--steps", "2", "--warmup", "1"])
+    assert bench.main() == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "GB/s"
+    assert line["value"] > 0 and line["higher_is_better"] is True and line["steps"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0

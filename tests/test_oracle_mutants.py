@@ -70,22 +70,33 @@ def _failing_pins(lib_path):
     return json.loads(res.stdout.strip().splitlines()[-1])
 
 
-def test_runner_accepts_the_real_oracle(tmp_path):
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Build every mutant (and the unmodified source as a control) and run the pins on each, eight child
+    processes at a time; returns {name: failing pins}."""
+    from concurrent.futures import ThreadPoolExecutor
+    d = tmp_path_factory.mktemp("mutants")
+    src = open(SRC).read()
+    libs = {"__control__": str(d / "lib_control.so")}
+    oracle.build(SRC, libs["__control__"])
+    for name, (old, new) in MUTANTS.items():
+        assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+        path = d / f"{name}.c"
+        path.write_text(src.replace(old, new))
+        libs[name] = str(d / f"lib_{name}.so")
+        oracle.build(str(path), libs[name])
+    with ThreadPoolExecutor(max_workers=8) as ex:
+        futures = {name: ex.submit(_failing_pins, lib) for name, lib in libs.items()}
+        return {name: f.result() for name, f in futures.items()}
+
+
+def test_runner_accepts_the_real_oracle(mutant_results):
     """Control: the unmodified source, built the same way, passes every pin in the runner."""
-    lib = str(tmp_path / "libpa_oracle_control.so")
-    oracle.build(SRC, lib)
-    assert _failing_pins(lib) == []
+    assert mutant_results["__control__"] == []
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_mutant_is_caught(name, tmp_path):
-    old, new = MUTANTS[name]
-    src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
-    mutated = tmp_path / "pa_oracle_mutant.c"
-    mutated.write_text(src.replace(old, new))
-    lib = str(tmp_path / "libpa_oracle_mutant.so")
-    oracle.build(str(mutated), lib)
-    failed = _failing_pins(lib)
+def test_mutant_is_caught(name, mutant_results):
+    failed = mutant_results[name]
     assert failed, f"mutant {name} passes every pin"
     print(f"{name}: caught by {failed}")
