@@ -79,19 +79,28 @@ int heads_per_unit(int group) {
 #ifndef PA_STAGES
 #define PA_STAGES 2
 #endif
-#ifndef PA_CHUNKS_PER_WARP
-#define PA_CHUNKS_PER_WARP 8
+// Balanced split (see ChunkPlan): per-mille share of each warp's tiles in its
+// static first chunk, and queued chunks per warp for the rest of the stream.
+// Measured on B200 (Llama-2, long-context, GQA and shared-prefix batches):
+// uniform chunks are best -- about 8 per warp for the CUDA-core kernel (fine
+// tail balancing), 1 per warp for the tensor-core kernel, whose cut pieces
+// carry several heads to merge; a large static first chunk loses more to
+// per-warp speed differences than it saves in merging.
+#ifndef PA_STATIC_PERMILLE
+#define PA_STATIC_PERMILLE 0
 #endif
-#ifndef PA_MMA_CHUNKS_PER_WARP
-#define PA_MMA_CHUNKS_PER_WARP 1
+#ifndef PA_TAIL_CHUNKS
+#define PA_TAIL_CHUNKS 8
+#endif
+#ifndef PA_MMA_STATIC_PERMILLE
+#define PA_MMA_STATIC_PERMILLE 0
+#endif
+#ifndef PA_MMA_TAIL_CHUNKS
+#define PA_MMA_TAIL_CHUNKS 1
 #endif
 constexpr int kWarps = PA_WARPS, kStages = PA_STAGES;
-// Balanced split: stream chunks per resident warp.  Measured on B200: the
-// CUDA-core kernel gains from several (fine tail balancing); the tensor-core
-// kernel, whose cut pieces carry up to 8 heads each to merge, prefers one.
-constexpr int kChunksPerWarp = PA_CHUNKS_PER_WARP;
-constexpr int kMmaChunksPerWarp = PA_MMA_CHUNKS_PER_WARP;
-int chunks_per_warp(int group) { return uses_mma(group) ? kMmaChunksPerWarp : kChunksPerWarp; }
+int static_permille(int group) { return uses_mma(group) ? PA_MMA_STATIC_PERMILLE : PA_STATIC_PERMILLE; }
+int tail_chunks(int group) { return uses_mma(group) ? PA_MMA_TAIL_CHUNKS : PA_TAIL_CHUNKS; }
 
 // Launches `kernel` with programmatic stream serialisation allowed: it may start
 // while the previous kernel in the stream finishes, and waits for it on the
@@ -219,7 +228,7 @@ int plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, i
   lp->grid = dtype == 0 ? 0 : sms * (dtype == PA_BFLOAT16 ? occ_bf16 : occ_f16);
   lp->chunk_tiles = partition_tokens / pa::TILE;
   if (lp->chunk_tiles == 0) {
-    lp->max_chunks = ws_warps * chunks_per_warp(group);
+    lp->max_chunks = ws_warps * (1 + tail_chunks(group)) + 1;
   } else {
     const long long per_seq = ((long long)max_context_len + pa::TILE - 1) / pa::TILE;
     const long long total = (long long)num_seqs * num_kv_heads * (group / G) * per_seq;
@@ -477,7 +486,8 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   a.n_chunks = group / G;
   a.chunk_tiles = lp.chunk_tiles;
   a.split_warps = lp.grid * kWarps;
-  a.chunks_per_warp = chunks_per_warp(group);
+  a.static_permille = static_permille(group);
+  a.tail_chunks_per_warp = tail_chunks(group);
   a.epoch = next_epoch();
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);

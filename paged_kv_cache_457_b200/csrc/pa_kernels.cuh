@@ -150,7 +150,8 @@ struct DecodeArgs {
   int heads_per_unit;  // query heads per head chunk (group / n_chunks)
   int chunk_tiles;     // tiles per chunk; 0: total tiles / split_warps
   int split_warps;     // warps in the split kernel's grid
-  int chunks_per_warp; // balanced split: target chunks per warp (the first one static, the rest from the queue)
+  int static_permille;       // balanced split: share of each warp's tiles in its static first chunk (per mille)
+  int tail_chunks_per_warp;  // balanced split: queued chunks per warp for the rest of the stream
   unsigned epoch;      // non-zero, different for every call
 };
 
@@ -197,20 +198,44 @@ __device__ __forceinline__ void build_tile_prefix(const DecodeArgs &a, int *pt, 
 
 constexpr int MIN_CHUNK_TILES = 4;  // never cut the stream finer than this (>= ring depth)
 
+// How the tile stream is cut.  The first `n1` chunks (one per warp of the
+// split kernel) hold `c1` tiles each; the rest of the stream is cut into
+// chunks of `c2` tiles, handed out through the queue.  With the balanced
+// split, c1 covers static_permille / 1000 of each warp's share and the tail
+// gives every warp about tail_chunks_per_warp more chunks; with a fixed
+// chunk length c1 = c2.  Boundaries depend only on the stream length and
+// the arguments, so every kernel of the call computes the same ones.
 struct ChunkPlan {
-  long long total, chunk, count;
-  __device__ __forceinline__ int length(long long c) const { return (int)min(chunk, total - c * chunk); }
+  long long total, c1, c2, n1, count;
+  __device__ __forceinline__ long long start(long long c) const {
+    return c < n1 ? c * c1 : n1 * c1 + (c - n1) * c2;
+  }
+  __device__ __forceinline__ int length(long long c) const {
+    return (int)min(c < n1 ? c1 : c2, total - start(c));
+  }
+  __device__ __forceinline__ long long chunk_of(long long t) const {
+    return t < n1 * c1 ? t / c1 : n1 + (t - n1 * c1) / c2;
+  }
 };
 
-// Chunk length and count for a tile stream of tiles_per_head_chunk_set * head_chunks tiles.
 __device__ __forceinline__ ChunkPlan plan_chunks(const DecodeArgs &a, int tiles_per_head_chunk_set) {
   ChunkPlan p;
   p.total = (long long)tiles_per_head_chunk_set * a.num_kv_heads * a.n_chunks;
-  const long long target = (long long)a.split_warps * a.chunks_per_warp;
-  long long c = a.chunk_tiles > 0 ? a.chunk_tiles : (p.total + target - 1) / target;
-  c = max(c, (p.total + a.max_chunks - 1) / a.max_chunks);  // never more chunks than the workspace holds
-  p.chunk = max(c, (long long)MIN_CHUNK_TILES);
-  p.count = (p.total + p.chunk - 1) / p.chunk;
+  const long long W = a.split_warps;
+  if (a.chunk_tiles > 0) {
+    p.c1 = p.c2 = max((long long)a.chunk_tiles, (long long)MIN_CHUNK_TILES);
+  } else {
+    p.c1 = p.total * a.static_permille / 1000 / W;
+    p.c2 = max((long long)MIN_CHUNK_TILES, (p.total - W * p.c1 + W * a.tail_chunks_per_warp - 1) /
+                                                max(1LL, W * a.tail_chunks_per_warp));
+    if (p.c1 < MIN_CHUNK_TILES) p.c1 = p.c2;  // a small stream: uniform chunks
+  }
+  // never more chunks than the workspace holds
+  p.n1 = min(W, (p.total + p.c1 - 1) / p.c1);
+  long long rest = max(0LL, p.total - p.n1 * p.c1);
+  if (a.max_chunks > p.n1 && rest > 0)
+    p.c2 = max(p.c2, (rest + (a.max_chunks - p.n1) - 1) / (a.max_chunks - p.n1));
+  p.count = p.n1 + (rest + p.c2 - 1) / p.c2;
   return p;
 }
 
@@ -468,7 +493,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
     long long prod_c = cons_c;
     int prod_left = plan.length(prod_c);
     bool prod_done = false;
-    TilePos cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
+    TilePos cp = locate_tile(pt, S, HC, plan.start(cons_c));
     prod.start(cp);
     uint32_t issued = iter;  // tiles issued by this warp: the next goes to ring slot issued % STAGES
 
@@ -485,7 +510,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
         }
         prod_c = nc;
         prod_left = plan.length(nc);
-        prod.start(locate_tile(pt, S, HC, nc * plan.chunk));
+        prod.start(locate_tile(pt, S, HC, plan.start(nc)));
       }
       const uint32_t it = issued++;
       const int phys = prod.lookup(a, lane);
@@ -525,7 +550,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
         if (prod_c == cons_c) break;
         cons_c = prod_c;
         cons_left = plan.length(cons_c);
-        cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
+        cp = locate_tile(pt, S, HC, plan.start(cons_c));
         k = 0;
       }
       if (k == 0 || cp.j == 0) {  // a new piece: segment (cp.s, cp.hc) from tile cp.j on
@@ -714,12 +739,12 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
       const int gg = r - ch * G;
       const int nt = pt1 - pt0;
       const long long seg0 = (long long)pt0 * HC + (long long)(h * a.n_chunks + ch) * nt;
-      const long long c_first = seg0 / plan.chunk, c_last = (seg0 + nt - 1) / plan.chunk;
+      const long long c_first = plan.chunk_of(seg0), c_last = plan.chunk_of(seg0 + nt - 1);
       if (c_first == c_last) continue;  // one chunk held the whole segment: the split kernel wrote the row
       const int n = (int)(c_last - c_first + 1);
       auto piece_row = [&](int p) -> int {  // partial row of piece p (chunk c_first + p)
         const long long c = c_first + p;
-        const int slot = (p == 0 && seg0 > c * plan.chunk) ? 1 : 0;
+        const int slot = (p == 0 && seg0 > plan.start(c)) ? 1 : 0;
         return (int)((c * 2 + slot) * G + gg);
       };
       // pass 1: maximum and validity over all pieces; lane p keeps piece p of the first 32

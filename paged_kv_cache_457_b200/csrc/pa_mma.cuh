@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
     long long prod_c = cons_c;
     int prod_left = plan.length(prod_c);
     bool prod_done = false;
-    TilePos cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
+    TilePos cp = locate_tile(pt, S, HC, plan.start(cons_c));
     prod.start(cp);
     uint32_t issued = iter;  // tiles issued by this warp: the next goes to ring slot issued % STAGES
 
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
         }
         prod_c = nc;
         prod_left = plan.length(nc);
-        prod.start(locate_tile(pt, S, HC, nc * plan.chunk));
+        prod.start(locate_tile(pt, S, HC, plan.start(nc)));
       }
       const uint32_t it = issued++;
       const int phys = prod.lookup(a, lane);
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
         if (prod_c == cons_c) break;
         cons_c = prod_c;
         cons_left = plan.length(cons_c);
-        cp = locate_tile(pt, S, HC, cons_c * plan.chunk);
+        cp = locate_tile(pt, S, HC, plan.start(cons_c));
         k = 0;
       }
       if (k == 0 || cp.j == 0) {  // a new piece: segment (cp.s, cp.hc) from tile cp.j on
