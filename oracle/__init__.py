@@ -9,6 +9,9 @@ cited in ``pa_oracle.c``:
 
 * ``write_kv``  -- "4. vLLM核心机制", section 4.3 (each iteration yields the
   updated KV cache) with the page layout of section 4.2;
+* ``copy_blocks`` -- "4. vLLM核心机制", section 4.2 (a private copy of a shared
+  page before a sequence appends to it) and section 4.4 (pages moved to a CPU-side
+  pool and back on preemption);
 * ``decode``    -- "4. vLLM核心机制", section 4.2 (page table lookup, pages
   anywhere in the pool) and "vLLM：大型语言模型推理优化的革命性突破",
   section 2.1 (no copy, no padding: plain attention over the logical tokens).
@@ -70,6 +73,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_decode.restype = ctypes.c_int
     lib.oracle_decode.argtypes = [p, p, p, p, i64, p, i64, i64, i64, i64, i64, i64, ctypes.c_int,
                                   ctypes.c_double, p]
+    lib.oracle_copy_blocks.restype = ctypes.c_int
+    lib.oracle_copy_blocks.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64]
     lib.oracle_half_to_double.restype = ctypes.c_double
     lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
     lib.oracle_bf16_to_double.restype = ctypes.c_double
@@ -144,3 +149,27 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype:
     if rc != 0:
         raise ValueError(f"oracle_decode: {ERRORS.get(rc, rc)}")
     return out
+
+
+def copy_blocks(src_k, src_v, dst_k, dst_v, mapping, lib_path: str | None = None):
+    """Copy whole blocks (all heads, rows, dims) from the source pools to the destination pools.
+
+    mapping: int64 [n, 2] (source block, destination block); negative entries skip the pair.
+    Returns new destination arrays (the source and destination may be the same arrays: pairs
+    are applied in order, reading the pools as updated so far).
+    """
+    lib = _load(lib_path)
+    sk, sv = _u16(src_k, "src_k"), _u16(src_v, "src_v")
+    same = src_k is dst_k
+    dk, dv = _u16(dst_k, "dst_k").copy(), _u16(dst_v, "dst_v").copy()
+    if same:
+        sk, sv = dk, dv
+    m = np.ascontiguousarray(mapping, dtype=np.int64).reshape(-1, 2)
+    if sk.shape[1:] != dk.shape[1:]:
+        raise ValueError("pools differ in heads, block size or head dim")
+    nb_s, hkv, bs, d = sk.shape
+    rc = lib.oracle_copy_blocks(_ptr(sk), _ptr(sv), _ptr(dk), _ptr(dv), _ptr(m) if len(m) else None, len(m), hkv,
+                                bs, d, nb_s, dk.shape[0])
+    if rc != 0:
+        raise ValueError(f"oracle_copy_blocks: {ERRORS.get(rc, rc)}")
+    return dk, dv

@@ -185,3 +185,30 @@ done:
     free(K); free(V); free(z);
     return rc;
 }
+
+/*
+ * Block copy ([P3] section 4.2: pages of a shared prefix are named by several
+ * tables; a sequence about to append to a shared, partly filled page first
+ * gets a private copy of it -- copy-on-write -- and section 4.4: preemption
+ * moves a sequence's pages to a CPU-side pool and back).  For every pair i,
+ * block mapping[i][0] of the source pool is copied, all kv heads, rows and
+ * dims, to block mapping[i][1] of the destination pool (which may be the
+ * same pool).  A pair with a negative entry is skipped.  Pools:
+ * [num_blocks][num_kv_heads][block_size][head_dim] 2-byte elements.
+ */
+int oracle_copy_blocks(const uint16_t *src_k, const uint16_t *src_v, uint16_t *dst_k, uint16_t *dst_v,
+                       const int64_t *mapping, int64_t num_pairs, int64_t num_kv_heads, int64_t block_size,
+                       int64_t head_dim, int64_t src_blocks, int64_t dst_blocks) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || block_size <= 0 || head_dim <= 0) return ORACLE_ERR_ARG;
+    const int64_t per_block = num_kv_heads * block_size * head_dim;
+    for (int64_t i = 0; i < num_pairs; ++i) {
+        const int64_t src = mapping[2 * i], dst = mapping[2 * i + 1];
+        if (src < 0 || dst < 0) continue;
+        if (src >= src_blocks || dst >= dst_blocks) return ORACLE_ERR_BLOCK_ID;
+        for (int64_t e = 0; e < per_block; ++e) {
+            dst_k[dst * per_block + e] = src_k[src * per_block + e];
+            dst_v[dst * per_block + e] = src_v[src * per_block + e];
+        }
+    }
+    return ORACLE_OK;
+}

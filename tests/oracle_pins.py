@@ -434,6 +434,56 @@ def pin_zero_length(lib=None):
     _close(out[1], sdpa_reference(q[1], lk[1], lv[1], 0.125, "fp16"), 1e-12, "neighbour of L=0")
 
 
+def pin_copy_blocks_is_fancy_indexing(lib=None):
+    """Block copies equal numpy's fancy-index assignment (pairs with distinct destinations, none of
+    which is another pair's source); untouched blocks and skipped pairs change nothing."""
+    rng = np.random.default_rng(31)
+    nb, hkv, bs, d = 12, 3, 16, 64
+    k = rng.integers(0, 65536, size=(nb, hkv, bs, d), dtype=np.uint16)
+    v = rng.integers(0, 65536, size=(nb, hkv, bs, d), dtype=np.uint16)
+    pairs = np.array([[1, 7], [4, 2], [-1, 3], [9, 11], [5, -1]], dtype=np.int64)
+    k2, v2 = oracle.copy_blocks(k, v, k, v, pairs, lib)
+    want_k, want_v = k.copy(), v.copy()
+    live = pairs[(pairs >= 0).all(axis=1)]
+    want_k[live[:, 1]] = k[live[:, 0]]
+    want_v[live[:, 1]] = v[live[:, 0]]
+    assert np.array_equal(k2, want_k) and np.array_equal(v2, want_v)
+
+
+def pin_swap_round_trip(lib=None):
+    """Swapping blocks out to a second pool and back restores them bit for bit."""
+    rng = np.random.default_rng(32)
+    dev_k = rng.integers(0, 65536, size=(10, 2, 32, 128), dtype=np.uint16)
+    dev_v = rng.integers(0, 65536, size=(10, 2, 32, 128), dtype=np.uint16)
+    host_k = np.zeros((6, 2, 32, 128), dtype=np.uint16)
+    host_v = host_k.copy()
+    out_pairs = np.array([[3, 0], [8, 5], [0, 2]], dtype=np.int64)
+    host_k, host_v = oracle.copy_blocks(dev_k, dev_v, host_k, host_v, out_pairs, lib)
+    for s_, d_ in out_pairs:
+        assert np.array_equal(host_k[d_], dev_k[s_]) and np.array_equal(host_v[d_], dev_v[s_])
+    wiped_k, wiped_v = dev_k.copy(), dev_v.copy()
+    wiped_k[[3, 8, 0]] = 0
+    wiped_v[[3, 8, 0]] = 0
+    back_k, back_v = oracle.copy_blocks(host_k, host_v, wiped_k, wiped_v, out_pairs[:, ::-1].copy(), lib)
+    assert np.array_equal(back_k, dev_k) and np.array_equal(back_v, dev_v)
+
+
+def pin_copy_on_write_decode(lib=None):
+    """A sequence that reads a private copy of a shared block decodes exactly as through the shared one."""
+    rng = np.random.default_rng(33)
+    q, lk, lv = random_case(rng, [40], 4, 2, 64, "fp16")
+    kc, tables = paged(lk, 16, 8, np.random.default_rng(34))
+    vc, _ = paged(lv, 16, 8, np.random.default_rng(34))
+    used = set(tables[0, :3].tolist())
+    spare = next(b for b in range(8) if b not in used)
+    kc2, vc2 = oracle.copy_blocks(kc, vc, kc, vc, np.array([[tables[0, 2], spare]], np.int64), lib)
+    t2 = tables.copy()
+    t2[0, 2] = spare
+    a = oracle.decode(q, kc, vc, tables, np.array([40], np.int32), 0.125, "fp16", lib)
+    b = oracle.decode(q, kc2, vc2, t2, np.array([40], np.int32), 0.125, "fp16", lib)
+    assert np.array_equal(a, b)
+
+
 ALL_PINS = [
     pin_widen_fp16,
     pin_widen_bf16,
@@ -454,4 +504,7 @@ ALL_PINS = [
     pin_write_kv_scatter,
     pin_write_then_decode_single,
     pin_zero_length,
+    pin_copy_blocks_is_fancy_indexing,
+    pin_swap_round_trip,
+    pin_copy_on_write_decode,
 ]

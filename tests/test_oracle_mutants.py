@@ -39,6 +39,11 @@ MUTANTS = {
     "write_head_stride": ("int64_t dst = ((block * num_kv_heads + h) * block_size + row) * head_dim + i;",
                           "int64_t dst = ((block * num_kv_heads) * block_size + row) * head_dim + i;"),
     "write_negative_slots": ("if (slot < 0) continue;", "if (slot < 0) slot = 0;"),
+    "copy_swaps_direction": ("dst_k[dst * per_block + e] = src_k[src * per_block + e];",
+                             "dst_k[src * per_block + e] = src_k[dst * per_block + e];"),
+    "copy_skips_v": ("            dst_v[dst * per_block + e] = src_v[src * per_block + e];\n", ""),
+    "copy_half_block": ("const int64_t per_block = num_kv_heads * block_size * head_dim;",
+                        "const int64_t per_block = block_size * head_dim;"),
     "zero_length_garbage": ("for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;\n            if (L == 0) continue;",
                             "if (L == 0) { o[0] = 1.0; continue; }\n            for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;"),
 }
