@@ -36,6 +36,14 @@ SEEDS = {"tiny_decode": 1, "llama2_7b_decode": 2, "gqa_llama3_decode": 3, "long_
          "shared_prefix_step": 5}
 
 
+# Block operations on a Llama-2-7B-shaped pool (32 kv heads, 16-token blocks,
+# head_dim 128, fp16: 128 KiB per block and cache).  copy_blocks is the
+# copy-on-write copy inside the device pool; swap_out / swap_in move blocks to
+# and from a pinned host pool (preemption).
+BLOCK_OPS = {"copy_blocks": 2048, "swap_out": 1024, "swap_in": 1024}
+BLOCK_POOL = {"num_blocks": 8192, "num_kv_heads": 32, "block_size": 16, "head_dim": 128, "dtype": "fp16"}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -43,6 +51,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.NAMED))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--op", default="decode", choices=["decode"] + sorted(BLOCK_OPS),
+                    help="decode step (default) or one of the block operations")
+    ap.add_argument("--pairs", type=int, default=None, help="block pairs per step (block operations)")
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -240,10 +251,191 @@ def run_reference(args):
     return 0
 
 
+def block_op_pairs(op: str, pairs: int, num_blocks: int, host_blocks: int, seed: int):
+    """(source, destination) pairs: distinct destinations, none of them a source of another pair."""
+    rng = np.random.default_rng(seed)
+    if op == "copy_blocks":
+        ids = rng.permutation(num_blocks)[: 2 * pairs]
+        return np.stack([ids[:pairs], ids[pairs:]], axis=1).astype(np.int64)
+    dev = rng.permutation(num_blocks)[:pairs]
+    host = rng.permutation(host_blocks)[:pairs]
+    pair = (dev, host) if op == "swap_out" else (host, dev)
+    return np.stack(pair, axis=1).astype(np.int64)
+
+
+def oracle_copy_rate(op: str, seconds: float):
+    """The oracle's block copy on host arrays: GB/s of block bytes moved (K and V), bounded sample."""
+    import oracle
+    g = BLOCK_POOL
+    nb, pairs = 256, 64
+    rng = np.random.default_rng(17)
+    shape = (nb, g["num_kv_heads"], g["block_size"], g["head_dim"])
+    k = rng.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+    v = rng.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+    m = block_op_pairs("copy_blocks", pairs, nb, nb, 3)
+    per_pair = 2 * int(np.prod(shape[1:])) * 2
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.copy_blocks(k, v, k, v, m)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    secs = time.perf_counter() - t0
+    return n * pairs * per_pair / secs / 1e9, f"{n} calls of {pairs} pairs on a {nb}-block host pool, {secs:.1f} s"
+
+
+def run_block_op(args):
+    """Times copy_blocks / swap_out / swap_in through the C ABI; prints one JSON line."""
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_457_b200 as pa
+
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    pa.load_library()
+    g = BLOCK_POOL
+    op = args.op
+    pairs = args.pairs or BLOCK_OPS[op]
+    nb = args.num_blocks or g["num_blocks"]
+    shape = (g["num_kv_heads"], g["block_size"], g["head_dim"])
+    block_bytes = int(np.prod(shape)) * 2
+    gen = torch.Generator(device=device).manual_seed(100 + rank)
+    k_cache = torch.randint(-32768, 32767, (nb,) + shape, dtype=torch.int16, device=device, generator=gen)
+    v_cache = torch.randint(-32768, 32767, (nb,) + shape, dtype=torch.int16, device=device, generator=gen)
+    k_cache, v_cache = k_cache.view(torch.float16), v_cache.view(torch.float16)
+    host_blocks = pairs
+    m_np = block_op_pairs(op, pairs, nb, host_blocks, 7 + rank)
+    mapping = torch.from_numpy(m_np).to(device)
+    if op == "copy_blocks":
+        call = lambda mp: pa.copy_blocks(k_cache, v_cache, mp)  # noqa: E731
+        host_k = host_v = None
+    else:
+        host_k = torch.empty((host_blocks,) + shape, dtype=torch.float16, pin_memory=True)
+        host_v = torch.empty((host_blocks,) + shape, dtype=torch.float16, pin_memory=True)
+        if op == "swap_out":
+            call = lambda mp: pa.swap_blocks(k_cache, v_cache, host_k, host_v, mp)  # noqa: E731
+        else:
+            call = lambda mp: pa.swap_blocks(host_k, host_v, k_cache, v_cache, mp, device=device)  # noqa: E731
+    moved = 2 * pairs * block_bytes  # K and V blocks per step
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device).start()
+    for _ in range(args.warmup):
+        call(mapping)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = pa.launch_count()
+    wall0 = time.perf_counter()
+    e0.record()
+    for _ in range(args.steps):
+        call(mapping)
+    e1.record()
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    launches = pa.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+
+    # End to end: the mapping comes from pinned host memory each step, the status word goes back.
+    host_map = torch.from_numpy(m_np).pin_memory()
+    status_host = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+    dmap = torch.empty_like(mapping)
+
+    def e2e_step():
+        dmap.copy_(host_map, non_blocking=True)
+        call(dmap)
+        status_host.copy_(torch.zeros(1, dtype=torch.int32, device=device), non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / args.steps
+
+    # The link's own rate for the swap legs: one contiguous pinned copy of the same bytes.
+    link = None
+    if op != "copy_blocks":
+        flat_dev = k_cache.view(-1)[: moved // 2]
+        flat_host = torch.empty(moved // 2, dtype=torch.float16, pin_memory=True)
+        for _ in range(3):
+            (flat_host.copy_(flat_dev, non_blocking=True) if op == "swap_out"
+             else flat_dev.copy_(flat_host, non_blocking=True))
+        torch.cuda.synchronize()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record()
+        for _ in range(args.steps):
+            (flat_host.copy_(flat_dev, non_blocking=True) if op == "swap_out"
+             else flat_dev.copy_(flat_host, non_blocking=True))
+        c1.record()
+        torch.cuda.synchronize()
+        link = (moved // 2 * 2) / (c0.elapsed_time(c1) / args.steps / 1e3) / 1e9
+    status = pa.device_status()
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, sample = oracle_copy_rate(op, min(args.cpu_sample_seconds, 5.0))
+        cpu = {"value": round(rate, 3), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample}
+    if rank == 0:
+        value = world * moved / (ms / 1e3) / 1e9
+        if op == "copy_blocks":
+            peak, peak_kind = measured_peak()
+            achieved = 2 * moved / (ms / 1e3) / 1e9  # read + write, as the copy peak counts them
+            roof = {"bound": "hbm", "kernel": "copy_blocks_kernel", "achieved": round(achieved, 1),
+                    "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                    "traffic": None, "algorithmic_bytes": 2 * moved, "ms_per_launch": round(ms, 5)}
+        else:
+            achieved = moved / (ms / 1e3) / 1e9
+            roof = {"bound": "host link", "kernel": "copy_blocks_kernel", "achieved": round(achieved, 1),
+                    "peak": round(link, 1), "peak_kind": "measured in this run: one contiguous pinned "
+                    + ("device-to-host" if op == "swap_out" else "host-to-device") + " copy of the same bytes",
+                    "unit": "GB/s", "frac": round(achieved / link, 4), "traffic": None,
+                    "algorithmic_bytes": moved, "ms_per_launch": round(ms, 5)}
+        line = {
+            "metric": f"{op} block bytes moved GB/s, 1×B200", "value": round(value, 2), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
+            "data": "synthetic",
+            "config": {"workload": f"{op}: {pairs} block pairs, Llama-2-7B pool geometry",
+                       "num_blocks": nb, "num_kv_heads": g["num_kv_heads"], "block_size": g["block_size"],
+                       "head_dim": g["head_dim"], "storage_dtype": g["dtype"], "pairs": pairs,
+                       "bytes_moved_per_step": moved, "parallelism": f"dp{world} (independent pools per GPU)",
+                       "l2": f"no flush: {moved / 2**20:.0f} MiB moved per step, larger than the 126 MB L2"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": round(world * moved / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(m_np.nbytes), "d2h_bytes_per_step": 4,
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": int(launches), "clocks": sampler.summary(wall0, wall1), "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op != "decode":
+        return run_block_op(args)
 
     import torch
     import torch.distributed as dist

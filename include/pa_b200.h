@@ -60,6 +60,7 @@ extern "C" {
 #define PA_ERR_PARTITION (-8)   /* partition_tokens negative or not a multiple of 16 */
 #define PA_ERR_CUDA (-9)        /* a CUDA runtime call failed; see pa_last_cuda_error() */
 #define PA_ERR_STATIC_WORKSPACE (-10) /* the problem needs more scratch than PA_STATIC_WORKSPACE_BYTES */
+#define PA_ERR_ADDRESS (-11)    /* a pointer is neither this device's memory nor pinned host memory mapped for it */
 
 /* Size of the fixed scratch array behind pa_decode_static_workspace (32 MiB). */
 #define PA_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
@@ -152,6 +153,41 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
               int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int64_t num_blocks,
               int32_t block_table_stride, int32_t max_context_len, int64_t q_seq_stride, int64_t out_seq_stride,
               int32_t partition_tokens, int32_t dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * pa_copy_blocks -- copy whole blocks inside one pair of caches: for every
+ * pair i, block block_mapping[i][0] is copied (all kv heads, rows and dims, K
+ * and V) to block block_mapping[i][1].  This is the copy a sequence needs
+ * before it appends to a block it shares with others (a prefix page named
+ * by several tables, "4. vLLM核心机制" section 4.2): it gets a private copy
+ * first (copy-on-write).
+ *   block_mapping  int64 [num_pairs][2], 8-byte aligned, in device memory
+ *                  or pinned host memory (checked as for pa_swap_blocks).
+ * A pair with a negative entry is skipped; an entry >= num_blocks is skipped
+ * and sets PA_DEV_ERR_BLOCK_ID.  Destinations must be distinct and must not
+ * be the source of another pair (pairs run concurrently).  Bit-exact copy.
+ */
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int64_t num_pairs,
+                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int64_t num_blocks, void *stream);
+
+/*
+ * pa_swap_blocks -- copy whole blocks from one pool (src_k, src_v with
+ * src_num_blocks blocks) to another (dst_k, dst_v with dst_num_blocks), with
+ * the same layout.  Either pool may be pinned host memory (reached through
+ * unified addressing): this moves a preempted sequence's pages to a
+ * CPU-side pool and back ("4. vLLM核心机制" section 4.4).  block_mapping
+ * pairs are (source block, destination block), device-accessible; rules as
+ * for pa_copy_blocks (entries checked against their own pool's size).
+ * Every pointer (pools and mapping) is checked with the runtime before the
+ * launch: device memory of the current device and pinned host memory are
+ * accepted (host pointers are translated to their device addresses);
+ * anything else (pageable host memory, another device's memory) returns
+ * PA_ERR_ADDRESS with nothing launched.  Host-side pools move over the host
+ * link, so a swap runs at that link's bandwidth.
+ */
+int pa_swap_blocks(const void *src_k, const void *src_v, void *dst_k, void *dst_v, const int64_t *block_mapping,
+                   int64_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                   int64_t src_num_blocks, int64_t dst_num_blocks, void *stream);
 
 /*
  * pa_get_device_status -- wait for `stream`, then copy the current device's

@@ -24,7 +24,7 @@ import threading
 import torch
 
 __all__ = [
-    "PagedAttentionError", "write_kv", "decode", "decode_workspace_size",
+    "PagedAttentionError", "write_kv", "decode", "decode_workspace_size", "copy_blocks", "swap_blocks",
     "device_status", "launch_count", "debug_wait_timeout", "library_path", "load_library", "EXPORTED_SYMBOLS",
     "DEV_ERR_BLOCK_ID", "DEV_ERR_CONTEXT", "DEV_ERR_CONTEXT_HINT", "DEV_ERR_SLOT", "DEV_ERR_TIMEOUT",
 ]
@@ -45,7 +45,7 @@ _DTYPES = {torch.float16: 1, torch.bfloat16: 2}
 EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_decode_workspace_size", "pa_decode",
     "pa_get_device_status", "pa_status_string", "pa_last_cuda_error", "pa_launch_count",
-    "pa_debug_wait_timeout", "pa_version", "pa_decode_static_workspace",
+    "pa_debug_wait_timeout", "pa_version", "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
 )
 
 
@@ -89,6 +89,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_decode_static_workspace.restype = ctypes.c_int
         lib.pa_decode_static_workspace.argtypes = [vp, vp, vp, vp, vp, f32, vp, i32, i32, i32, i32, i32, i64, i32,
                                                    i32, i64, i64, i32, i32, vp]
+        lib.pa_copy_blocks.restype = ctypes.c_int
+        lib.pa_copy_blocks.argtypes = [vp, vp, vp, i64, i32, i32, i32, i64, vp]
+        lib.pa_swap_blocks.restype = ctypes.c_int
+        lib.pa_swap_blocks.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, i64, vp]
         lib.pa_version.restype = i32
         lib.pa_version.argtypes = []
         if path is None:
@@ -211,6 +215,44 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
                        workspace.numel() * workspace.element_size() if workspace is not None else 0, stream)
     _check(rc, "pa_decode")
     return out
+
+
+def _mapping(block_mapping: torch.Tensor, device: torch.device) -> torch.Tensor:
+    if block_mapping.dtype != torch.int64 or block_mapping.dim() != 2 or block_mapping.shape[1] != 2 \
+            or not block_mapping.is_contiguous():
+        raise PagedAttentionError("block_mapping must be a contiguous int64 [n, 2] tensor")
+    if not block_mapping.is_cuda and not block_mapping.is_pinned():
+        raise PagedAttentionError("block_mapping must be on the GPU or in pinned host memory")
+    return block_mapping
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: torch.Tensor) -> None:
+    """Copy block block_mapping[i, 0] to block block_mapping[i, 1] inside the caches (copy-on-write)."""
+    dev = k_cache.device
+    _need_cuda("k_cache", k_cache, dev)
+    _need_cuda("v_cache", v_cache, dev)
+    nb, hkv, bs, d = _cache_geometry(k_cache, v_cache)
+    m = _mapping(block_mapping, dev)
+    rc = load_library().pa_copy_blocks(k_cache.data_ptr(), v_cache.data_ptr(), m.data_ptr(), int(m.shape[0]), hkv, d,
+                                       bs, nb, _stream(dev))
+    _check(rc, "pa_copy_blocks")
+
+
+def swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor, dst_v: torch.Tensor,
+                block_mapping: torch.Tensor, device: torch.device | None = None) -> None:
+    """Copy blocks between two pools of the same layout; either may be pinned host memory."""
+    for name, t in (("src_k", src_k), ("src_v", src_v), ("dst_k", dst_k), ("dst_v", dst_v)):
+        if not (t.is_cuda or t.is_pinned()):
+            raise PagedAttentionError(f"{name} must be on the GPU or in pinned host memory")
+    dev = device or next((t.device for t in (src_k, dst_k) if t.is_cuda), torch.device("cuda", torch.cuda.current_device()))
+    snb, hkv, bs, d = _cache_geometry(src_k, src_v)
+    dnb = _cache_geometry(dst_k, dst_v)
+    if dnb[1:] != (hkv, bs, d) or src_k.dtype != dst_k.dtype:
+        raise PagedAttentionError("pools must share heads, block size, head dim and dtype")
+    m = _mapping(block_mapping, dev)
+    rc = load_library().pa_swap_blocks(src_k.data_ptr(), src_v.data_ptr(), dst_k.data_ptr(), dst_v.data_ptr(),
+                                       m.data_ptr(), int(m.shape[0]), hkv, d, bs, snb, dnb[0], _stream(dev))
+    _check(rc, "pa_swap_blocks")
 
 
 def device_status(clear: bool = True, device: torch.device | None = None) -> int:

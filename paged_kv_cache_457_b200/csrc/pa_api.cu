@@ -59,6 +59,36 @@ int current_sms(int *sms_out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The address at which the current device reaches `p`: device memory of this
+// device as is, pinned (page-locked, mapped) host memory through its device
+// alias.  Anything else would fault inside a kernel, so it is refused here.
+int device_view(const void *p, const void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record(e);
+  cudaPointerAttributes at{};
+  e = cudaPointerGetAttributes(&at, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_ADDRESS;
+  }
+  switch (at.type) {
+    case cudaMemoryTypeDevice:
+      if (at.device != dev) return PA_ERR_ADDRESS;
+      *out = p;
+      return PA_OK;
+    case cudaMemoryTypeManaged:
+      *out = p;
+      return PA_OK;
+    case cudaMemoryTypeHost:
+      if (!at.devicePointer) return PA_ERR_ADDRESS;
+      *out = at.devicePointer;
+      return PA_OK;
+    default:
+      return PA_ERR_ADDRESS;
+  }
+}
+
 // Query heads handled together by one head chunk (the K/V tiles are read once
 // for all of them).  Groups of 1 or 2 run on the CUDA-core kernel; larger
 // groups run on the tensor-core kernel, whose chunks take up to 8 query heads
@@ -526,6 +556,7 @@ const char *pa_status_string(int32_t status) {
     case PA_ERR_WORKSPACE: return "workspace missing, smaller than pa_decode_workspace_size() or misaligned";
     case PA_ERR_PARTITION: return "partition_tokens must be 0 or a positive multiple of 16";
     case PA_ERR_CUDA: return "a CUDA runtime call failed (see pa_last_cuda_error)";
+    case PA_ERR_ADDRESS: return "a pointer is neither this device's memory nor mapped pinned host memory";
     case PA_ERR_STATIC_WORKSPACE:
       return "the problem needs more split-context scratch than the library's fixed 32 MiB array; "
              "use pa_decode with a caller workspace or a larger partition_tokens";
@@ -565,6 +596,50 @@ int pa_decode_static_workspace(const void *q, const void *k_cache, const void *v
   return pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, num_seqs, num_q_heads, num_kv_heads,
                    head_dim, block_size, num_blocks, block_table_stride, max_context_len, q_seq_stride,
                    out_seq_stride, partition_tokens, dtype, scratch, PA_STATIC_WORKSPACE_BYTES, stream);
+}
+
+int pa_swap_blocks(const void *src_k, const void *src_v, void *dst_k, void *dst_v, const int64_t *block_mapping,
+                   int64_t num_pairs, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                   int64_t src_num_blocks, int64_t dst_num_blocks, void *stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || src_num_blocks <= 0 || dst_num_blocks <= 0) return PA_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!src_k || !src_v || !dst_k || !dst_v || !block_mapping) return PA_ERR_NULL;
+  if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v) ||
+      (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+    return PA_ERR_ALIGN;
+  const void *view[5];
+  const void *ptrs[5] = {src_k, src_v, dst_k, dst_v, block_mapping};
+  for (int i = 0; i < 5; ++i) {
+    const int rc = device_view(ptrs[i], &view[i]);
+    if (rc != PA_OK) return rc;
+  }
+  int sms = 0;
+  int rc = current_sms(&sms);
+  if (rc != PA_OK) return rc;
+  pa::CopyArgs a;
+  a.src_k = static_cast<const uint4 *>(view[0]);
+  a.src_v = static_cast<const uint4 *>(view[1]);
+  a.dst_k = static_cast<uint4 *>(const_cast<void *>(view[2]));
+  a.dst_v = static_cast<uint4 *>(const_cast<void *>(view[3]));
+  a.mapping = static_cast<const int64_t *>(view[4]);
+  a.num_pairs = num_pairs;
+  a.chunks_per_block = (long long)num_kv_heads * block_size * head_dim * 2 / 16;
+  a.src_blocks = src_num_blocks;
+  a.dst_blocks = dst_num_blocks;
+  const long long work = num_pairs * 2 * ((a.chunks_per_block + 3) / 4);
+  const int grid = (int)std::max(1LL, std::min<long long>((work + 255) / 256, (long long)sms * 8));
+  cudaError_t e = launch_pdl(pa::copy_blocks_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), a);
+  if (e != cudaSuccess) return record(e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int64_t num_pairs,
+                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int64_t num_blocks, void *stream) {
+  return pa_swap_blocks(k_cache, v_cache, k_cache, v_cache, block_mapping, num_pairs, num_kv_heads, head_dim,
+                        block_size, num_blocks, num_blocks, stream);
 }
 
 int32_t pa_version(void) { return 100; }
