@@ -27,6 +27,7 @@ __all__ = [
     "PagedAttentionError", "write_kv", "decode", "decode_workspace_size", "copy_blocks", "swap_blocks",
     "device_status", "launch_count", "debug_wait_timeout", "library_path", "load_library", "EXPORTED_SYMBOLS",
     "DEV_ERR_BLOCK_ID", "DEV_ERR_CONTEXT", "DEV_ERR_CONTEXT_HINT", "DEV_ERR_SLOT", "DEV_ERR_TIMEOUT",
+    "BlockManager", "BlockManagerError", "DecodeStepPlan",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -46,6 +47,10 @@ EXPORTED_SYMBOLS = (
     "pa_write_kv", "pa_decode_workspace_size", "pa_decode",
     "pa_get_device_status", "pa_status_string", "pa_last_cuda_error", "pa_launch_count",
     "pa_debug_wait_timeout", "pa_version", "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
+    "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_device_blocks", "pa_bm_num_free_host_blocks",
+    "pa_bm_ref_count", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_num_tokens",
+    "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step",
+    "pa_bm_swap_out", "pa_bm_swap_in",
 )
 
 
@@ -95,6 +100,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_swap_blocks.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, i64, vp]
         lib.pa_version.restype = i32
         lib.pa_version.argtypes = []
+        from .block_manager import bind as _bind_block_manager
+        _bind_block_manager(lib)
         if path is None:
             _lib = lib
         return lib
@@ -271,3 +278,6 @@ def launch_count() -> int:
 def debug_wait_timeout(limit_ns: int = 10_000_000) -> None:
     dev = torch.device("cuda", torch.cuda.current_device())
     _check(load_library().pa_debug_wait_timeout(int(limit_ns), _stream(dev)), "pa_debug_wait_timeout")
+
+
+from .block_manager import BlockManager, BlockManagerError, DecodeStepPlan  # noqa: E402
