@@ -14,7 +14,10 @@ cited in ``pa_oracle.c``:
   pool and back on preemption);
 * ``decode``    -- "4. vLLM核心机制", section 4.2 (page table lookup, pages
   anywhere in the pool) and "vLLM：大型语言模型推理优化的革命性突破",
-  section 2.1 (no copy, no padding: plain attention over the logical tokens).
+  section 2.1 (no copy, no padding: plain attention over the logical tokens);
+* ``prefill``   -- "4. vLLM核心机制", section 4.3 (the prompt enters the cache
+  before decoding, possibly in pieces): causal attention of several new
+  tokens per sequence over the paged context.
 
 All pins (closed forms, invariants, library special cases, the page-table
 worked example) live in ``tests/test_oracle_pins.py``; no function here is
@@ -73,6 +76,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_decode.restype = ctypes.c_int
     lib.oracle_decode.argtypes = [p, p, p, p, i64, p, i64, i64, i64, i64, i64, i64, ctypes.c_int,
                                   ctypes.c_double, p]
+    lib.oracle_prefill.restype = ctypes.c_int
+    lib.oracle_prefill.argtypes = [p, p, p, p, i64, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_int,
+                                   ctypes.c_double, p]
     lib.oracle_copy_blocks.restype = ctypes.c_int
     lib.oracle_copy_blocks.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, i64]
     lib.oracle_half_to_double.restype = ctypes.c_double
@@ -173,3 +179,35 @@ def copy_blocks(src_k, src_v, dst_k, dst_v, mapping, lib_path: str | None = None
     if rc != 0:
         raise ValueError(f"oracle_copy_blocks: {ERRORS.get(rc, rc)}")
     return dk, dv
+
+
+def prefill(q, k_cache, v_cache, block_tables, query_start, context_lens, scale: float, dtype: str,
+            lib_path: str | None = None) -> np.ndarray:
+    """Exact (fp64) causal attention of each sequence's new tokens over its paged context.
+
+    q: uint16 [N, Hq, d] (N = query_start[-1]); query_start: int32 [S + 1], query_start[0] = 0;
+    context_lens: int32 [S], every token of the sequence including the new ones.  Returns
+    float64 [N, Hq, d].
+    """
+    lib = _load(lib_path)
+    q = _u16(q, "q")
+    kc = _u16(k_cache, "k_cache")
+    vc = _u16(v_cache, "v_cache")
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S = cl.shape[0]
+    N, hq, d = q.shape
+    nb, hkv, bs, d2 = kc.shape
+    if d2 != d or vc.shape != kc.shape:
+        raise ValueError("cache shapes do not match q")
+    if qs.shape != (S + 1,) or bt.ndim != 2 or bt.shape[0] != S or int(qs[-1]) != N:
+        raise ValueError("query_start must be [S + 1] ending at the number of query rows; block_tables [S, MB]")
+    out = np.zeros((N, hq, d), dtype=np.float64)
+    if S == 0 or N == 0:
+        return out
+    rc = lib.oracle_prefill(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), bt.shape[1], _ptr(qs), _ptr(cl), S, hq, hkv, d,
+                            bs, nb, DTYPE_CODES[dtype], float(scale), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_prefill: {ERRORS.get(rc, rc)}")
+    return out

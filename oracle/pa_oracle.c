@@ -103,14 +103,58 @@ int oracle_write_kv(const uint16_t *k, const uint16_t *v, uint16_t *k_cache, uin
 }
 
 /*
+ * Step 1 of both attention functions ([P3] section 4.2): the L logical tokens
+ * of one sequence and kv head h, gathered through its page-table row: token j
+ * lives in physical block table_row[j / block_size], row j % block_size.
+ * Writes contiguous K[L][d] and V[L][d].
+ */
+static void gather_rows(const uint16_t *k_cache, const uint16_t *v_cache, const int32_t *table_row, int64_t L,
+                        int64_t h, int64_t num_kv_heads, int64_t head_dim, int64_t block_size, int dtype,
+                        double *K, double *V) {
+    for (int64_t j = 0; j < L; ++j) {
+        int64_t p = table_row[j / block_size];
+        int64_t row = j % block_size;
+        const uint16_t *kr = k_cache + ((p * num_kv_heads + h) * block_size + row) * head_dim;
+        const uint16_t *vr = v_cache + ((p * num_kv_heads + h) * block_size + row) * head_dim;
+        for (int64_t i = 0; i < head_dim; ++i) {
+            K[j * head_dim + i] = widen(kr[i], dtype);
+            V[j * head_dim + i] = widen(vr[i], dtype);
+        }
+    }
+}
+
+/*
+ * Steps 2-4 for one query row qr over the first `count` gathered tokens
+ * ([P1] section 2.1: plain attention over the logical tokens):
+ *   z_j = scale * sum_i q[i] * K[j][i];  w_j = exp(z_j - max_j z_j);
+ *   o[i] += sum_j (w_j / sum_j w_j) * V[j][i].
+ * z is scratch of `count` doubles; o must hold zeros on entry.
+ */
+static void attend(const uint16_t *qr, const double *K, const double *V, int64_t count, int64_t head_dim,
+                   int dtype, double scale, double *z, double *o) {
+    for (int64_t j = 0; j < count; ++j) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < head_dim; ++i) acc += widen(qr[i], dtype) * K[j * head_dim + i];
+        z[j] = scale * acc;
+    }
+    double m = z[0];
+    for (int64_t j = 1; j < count; ++j)
+        if (z[j] > m) m = z[j];
+    double Z = 0.0;
+    for (int64_t j = 0; j < count; ++j) {
+        z[j] = exp(z[j] - m);
+        Z += z[j];
+    }
+    for (int64_t j = 0; j < count; ++j) {
+        double w = z[j] / Z;
+        for (int64_t i = 0; i < head_dim; ++i) o[i] += w * V[j * head_dim + i];
+    }
+}
+
+/*
  * Decode attention for one new query token per sequence.  For sequence s and
- * query head hq (kv head h):
- *   1. gather the L = context_lens[s] logical tokens through the page table:
- *      token j lives in physical block block_tables[s][j / block_size], row
- *      j % block_size ([P3] section 4.2), giving contiguous K[L][d], V[L][d];
- *   2. z_j = scale * sum_i q[i] * K[j][i];
- *   3. w_j = exp(z_j - max_j z_j),  Z = sum_j w_j;
- *   4. out[i] = sum_j (w_j / Z) * V[j][i]                    ([P1] section 2.1)
+ * query head hq (kv head h = hq / group), gather the L = context_lens[s]
+ * tokens (step 1) and attend over all of them (steps 2-4).
  * q: [num_seqs][num_q_heads][head_dim]; block_tables: [num_seqs][table_stride];
  * out: [num_seqs][num_q_heads][head_dim] doubles.
  */
@@ -145,38 +189,9 @@ int oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_
             double *o = out + (s * num_q_heads + hq) * head_dim;
             for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;
             if (L == 0) continue;
-            /* step 1: gather */
-            for (int64_t j = 0; j < L; ++j) {
-                int64_t p = block_tables[s * table_stride + j / block_size];
-                int64_t row = j % block_size;
-                const uint16_t *kr = k_cache + ((p * num_kv_heads + h) * block_size + row) * head_dim;
-                const uint16_t *vr = v_cache + ((p * num_kv_heads + h) * block_size + row) * head_dim;
-                for (int64_t i = 0; i < head_dim; ++i) {
-                    K[j * head_dim + i] = widen(kr[i], dtype);
-                    V[j * head_dim + i] = widen(vr[i], dtype);
-                }
-            }
-            /* step 2: scaled dot products */
-            const uint16_t *qr = q + (s * num_q_heads + hq) * head_dim;
-            for (int64_t j = 0; j < L; ++j) {
-                double acc = 0.0;
-                for (int64_t i = 0; i < head_dim; ++i) acc += widen(qr[i], dtype) * K[j * head_dim + i];
-                z[j] = scale * acc;
-            }
-            /* step 3: softmax weights */
-            double m = z[0];
-            for (int64_t j = 1; j < L; ++j)
-                if (z[j] > m) m = z[j];
-            double Z = 0.0;
-            for (int64_t j = 0; j < L; ++j) {
-                z[j] = exp(z[j] - m);
-                Z += z[j];
-            }
-            /* step 4: weighted sum of V rows */
-            for (int64_t j = 0; j < L; ++j) {
-                double w = z[j] / Z;
-                for (int64_t i = 0; i < head_dim; ++i) o[i] += w * V[j * head_dim + i];
-            }
+            gather_rows(k_cache, v_cache, block_tables + s * table_stride, L, h, num_kv_heads, head_dim,
+                        block_size, dtype, K, V);
+            attend(q + (s * num_q_heads + hq) * head_dim, K, V, L, head_dim, dtype, scale, z, o);
         }
         free(K); free(V); free(z);
         K = V = z = NULL;
@@ -211,4 +226,66 @@ int oracle_copy_blocks(const uint16_t *src_k, const uint16_t *src_v, uint16_t *d
         }
     }
     return ORACLE_OK;
+}
+
+/*
+ * Prefill / chunked prefill through the page table ([P3] section 4.3: the
+ * prompt's tokens enter the cache before decoding starts, and a long prompt
+ * may be processed in pieces across iterations).  Sequence s brings
+ * n = query_start[s+1] - query_start[s] new query tokens; its K/V rows for
+ * all L = context_lens[s] tokens, the new ones included, are already in the
+ * paged cache.  New token t sits at logical position pos = L - n + t and
+ * attends causally to tokens 0..pos: steps 1-4 of decode with the first
+ * pos + 1 gathered tokens.  With n = 1 this is exactly decode.
+ * q, out: [total_new_tokens][num_q_heads][head_dim], token-major.
+ */
+int oracle_prefill(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                   const int32_t *block_tables, int64_t table_stride, const int32_t *query_start,
+                   const int32_t *context_lens, int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads,
+                   int64_t head_dim, int64_t block_size, int64_t num_blocks, int dtype, double scale,
+                   double *out) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_q_heads % num_kv_heads != 0 || (dtype != 1 && dtype != 2))
+        return ORACLE_ERR_ARG;
+    if (num_seqs > 0 && query_start[0] != 0) return ORACLE_ERR_ARG;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t n = (int64_t)query_start[s + 1] - query_start[s];
+        int64_t L = context_lens[s];
+        if (n < 0) return ORACLE_ERR_ARG;
+        if (L < n || L > table_stride * block_size) return ORACLE_ERR_CONTEXT;
+        for (int64_t j = 0; j < L; j += block_size) {
+            int32_t p = block_tables[s * table_stride + j / block_size];
+            if (p < 0 || p >= num_blocks) return ORACLE_ERR_BLOCK_ID;
+        }
+    }
+    int64_t group = num_q_heads / num_kv_heads;
+    double *K = NULL, *V = NULL, *z = NULL;
+    int rc = ORACLE_OK;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t n = (int64_t)query_start[s + 1] - query_start[s];
+        int64_t L = context_lens[s];
+        if (n == 0) continue;
+        K = (double *)malloc((size_t)(L * head_dim) * sizeof(double));
+        V = (double *)malloc((size_t)(L * head_dim) * sizeof(double));
+        z = (double *)malloc((size_t)L * sizeof(double));
+        if (!K || !V || !z) { rc = ORACLE_ERR_NOMEM; goto done; }
+        for (int64_t h = 0; h < num_kv_heads; ++h) {
+            gather_rows(k_cache, v_cache, block_tables + s * table_stride, L, h, num_kv_heads, head_dim,
+                        block_size, dtype, K, V);
+            for (int64_t hq = h * group; hq < (h + 1) * group; ++hq) {
+                for (int64_t t = 0; t < n; ++t) {
+                    int64_t pos = L - n + t;
+                    int64_t tok = query_start[s] + t;
+                    double *o = out + (tok * num_q_heads + hq) * head_dim;
+                    for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;
+                    attend(q + (tok * num_q_heads + hq) * head_dim, K, V, pos + 1, head_dim, dtype, scale, z, o);
+                }
+            }
+        }
+        free(K); free(V); free(z);
+        K = V = z = NULL;
+    }
+done:
+    free(K); free(V); free(z);
+    return rc;
 }

@@ -484,6 +484,100 @@ def pin_copy_on_write_decode(lib=None):
     assert np.array_equal(a, b)
 
 
+def causal_reference(q_bits, k_rows, v_rows, scale, dtype):
+    """torch fp64 SDPA of n new tokens (q_bits [n, Hq, d]) over L contiguous rows ([L, Hkv, d]).
+
+    The new tokens are the last n of the L; token t may see rows 0..L-n+t (an explicit mask:
+    the causal diagonal ends at the bottom-right corner).
+    """
+    n, hq, _ = q_bits.shape
+    L, hkv, _ = k_rows.shape
+    q = torch.from_numpy(from_bits(q_bits, dtype)).permute(1, 0, 2).unsqueeze(0)
+    k = torch.from_numpy(from_bits(k_rows, dtype)).permute(1, 0, 2).unsqueeze(0).repeat_interleave(hq // hkv, 1)
+    v = torch.from_numpy(from_bits(v_rows, dtype)).permute(1, 0, 2).unsqueeze(0).repeat_interleave(hq // hkv, 1)
+    mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=scale)
+    return o[0].permute(1, 0, 2).numpy()
+
+
+def prefill_case(rng, shape, hq, hkv, d, bs, dtype, nb_extra=4):
+    """shape: [(L, n)] per sequence.  Returns q [N, Hq, d], logical rows, caches, tables, query_start, lens."""
+    lens = [L for L, _ in shape]
+    logical_k = [to_bits(rng.standard_normal((L, hkv, d)), dtype) for L in lens]
+    logical_v = [to_bits(rng.standard_normal((L, hkv, d)), dtype) for L in lens]
+    qs = np.concatenate([[0], np.cumsum([n for _, n in shape])]).astype(np.int32)
+    q = to_bits(rng.standard_normal((int(qs[-1]), hq, d)), dtype)
+    nb = sum(-(-L // bs) for L in lens) + nb_extra
+    kc, tables = paged(logical_k, bs, nb, np.random.default_rng(50), dtype=dtype)
+    vc, _ = paged(logical_v, bs, nb, np.random.default_rng(50), dtype=dtype)
+    return q, logical_k, logical_v, kc, vc, tables, qs, np.array(lens, np.int32)
+
+
+def pin_prefill_matches_library_causal(lib=None):
+    """Prompt and chunked-prompt rows of several sequences against torch fp64 SDPA with the causal mask."""
+    rng = np.random.default_rng(41)
+    cases = [  # [(L, n)], hq, hkv, d, bs, dtype
+        ([(1, 1), (16, 16), (17, 17), (40, 8), (100, 1), (70, 33)], 8, 2, 64, 16, "fp16"),
+        ([(33, 33), (64, 20), (5, 2)], 4, 4, 128, 32, "bf16"),
+    ]
+    for shape, hq, hkv, d, bs, dtype in cases:
+        q, lk, lv, kc, vc, tables, qs, lens = prefill_case(rng, shape, hq, hkv, d, bs, dtype)
+        scale = 1.0 / math.sqrt(d)
+        out = oracle.prefill(q, kc, vc, tables, qs, lens, scale, dtype, lib)
+        for s in range(len(shape)):
+            rows = slice(qs[s], qs[s + 1])
+            _close(out[rows], causal_reference(q[rows], lk[s], lv[s], scale, dtype), 1e-12,
+                   f"prefill (L, n) = {shape[s]}")
+
+
+def pin_prefill_first_token_is_v0(lib=None):
+    """A whole prompt: the token at position 0 sees only itself, so its output is V[0] exactly."""
+    rng = np.random.default_rng(42)
+    q, lk, lv, kc, vc, tables, qs, lens = prefill_case(rng, [(23, 23), (9, 9)], 6, 3, 64, 16, "fp16")
+    out = oracle.prefill(q, kc, vc, tables, qs, lens, 0.3, "fp16", lib)
+    for s in range(2):
+        want = from_bits(lv[s][0], "fp16").repeat(2, axis=0)  # 2 query heads per kv head
+        assert np.array_equal(out[qs[s]], want)
+
+
+def pin_prefill_chunked_equals_whole(lib=None):
+    """A prompt processed in two chunks (the second one over the cached first) equals one pass."""
+    rng = np.random.default_rng(43)
+    q, lk, lv, kc, vc, tables, qs, lens = prefill_case(rng, [(50, 50)], 4, 2, 64, 16, "bf16")
+    whole = oracle.prefill(q, kc, vc, tables, qs, lens, 0.125, "bf16", lib)
+    first = oracle.prefill(q[:30], kc, vc, tables, np.array([0, 30], np.int32), np.array([30], np.int32), 0.125,
+                           "bf16", lib)
+    second = oracle.prefill(q[30:], kc, vc, tables, np.array([0, 20], np.int32), np.array([50], np.int32), 0.125,
+                            "bf16", lib)
+    assert np.array_equal(np.concatenate([first, second]), whole)
+
+
+def pin_prefill_is_causal(lib=None):
+    """Rewriting the K/V rows after position p leaves the outputs of positions <= p unchanged."""
+    rng = np.random.default_rng(44)
+    q, lk, lv, kc, vc, tables, qs, lens = prefill_case(rng, [(48, 48)], 2, 2, 64, 16, "fp16")
+    a = oracle.prefill(q, kc, vc, tables, qs, lens, 0.125, "fp16", lib)
+    p = 29
+    lk2, lv2 = lk[0].copy(), lv[0].copy()
+    lk2[p + 1:] = to_bits(rng.standard_normal(lk2[p + 1:].shape), "fp16")
+    lv2[p + 1:] = to_bits(rng.standard_normal(lv2[p + 1:].shape), "fp16")
+    kc2, _ = paged([lk2], 16, tables.size + 4, np.random.default_rng(50))
+    vc2, _ = paged([lv2], 16, tables.size + 4, np.random.default_rng(50))
+    b = oracle.prefill(q, kc2, vc2, tables, qs, lens, 0.125, "fp16", lib)
+    assert np.array_equal(a[:p + 1], b[:p + 1])
+    assert not np.array_equal(a[p + 1:], b[p + 1:])
+
+
+def pin_prefill_one_new_token_is_decode(lib=None):
+    """One new token per sequence is the decode step: equal to the decode function bit for bit."""
+    rng = np.random.default_rng(45)
+    shape = [(1, 1), (37, 1), (64, 1), (65, 1)]
+    q, lk, lv, kc, vc, tables, qs, lens = prefill_case(rng, shape, 8, 2, 128, 32, "fp16")
+    a = oracle.prefill(q, kc, vc, tables, qs, lens, 0.1, "fp16", lib)
+    b = oracle.decode(q, kc, vc, tables, lens, 0.1, "fp16", lib)
+    assert np.array_equal(a, b)
+
+
 ALL_PINS = [
     pin_widen_fp16,
     pin_widen_bf16,
@@ -507,4 +601,9 @@ ALL_PINS = [
     pin_copy_blocks_is_fancy_indexing,
     pin_swap_round_trip,
     pin_copy_on_write_decode,
+    pin_prefill_matches_library_causal,
+    pin_prefill_first_token_is_v0,
+    pin_prefill_chunked_equals_whole,
+    pin_prefill_is_causal,
+    pin_prefill_one_new_token_is_decode,
 ]

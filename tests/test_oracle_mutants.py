@@ -18,17 +18,16 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.c")
 
 MUTANTS = {
     "row_uses_division": ("int64_t row = j % block_size;", "int64_t row = j / block_size;"),
-    "table_uses_modulo": ("block_tables[s * table_stride + j / block_size];\n                int64_t row",
-                          "block_tables[s * table_stride + j % block_size];\n                int64_t row"),
+    "table_uses_modulo": ("table_row[j / block_size];\n        int64_t row", "table_row[j % block_size];\n        int64_t row"),
     "gqa_modulo_grouping": ("int64_t h = hq / group;", "int64_t h = hq % num_kv_heads;"),
     "dropped_scale": ("z[j] = scale * acc;", "z[j] = acc;"),
     "softmax_sign": ("z[j] = exp(z[j] - m);", "z[j] = exp(m - z[j]);"),
     "no_max_shift": ("z[j] = exp(z[j] - m);", "z[j] = exp(z[j]);"),
     "dropped_normaliser": ("double w = z[j] / Z;", "double w = z[j];"),
     "k_v_swapped": ("K[j * head_dim + i] = widen(kr[i], dtype);", "K[j * head_dim + i] = widen(vr[i], dtype);"),
-    "query_of_kv_head": ("q + (s * num_q_heads + hq) * head_dim;", "q + (s * num_q_heads + h) * head_dim;"),
-    "last_token_dropped": ("for (int64_t j = 0; j < L; ++j) {\n                int64_t p",
-                           "for (int64_t j = 0; j < L - 1; ++j) {\n                int64_t p"),
+    "query_of_kv_head": ("attend(q + (s * num_q_heads + hq) * head_dim,", "attend(q + (s * num_q_heads + h) * head_dim,"),
+    "last_token_dropped": ("for (int64_t j = 0; j < L; ++j) {\n        int64_t p",
+                           "for (int64_t j = 0; j < L - 1; ++j) {\n        int64_t p"),
     "fp16_no_implicit_bit": ("ldexp((double)(f + 1024), e - 25)", "ldexp((double)f, e - 25)"),
     "fp16_bias_off_by_one": ("ldexp((double)(f + 1024), e - 25)", "ldexp((double)(f + 1024), e - 24)"),
     "fp16_subnormal_scale": ("ldexp((double)f, -24);", "ldexp((double)f, -25);"),
@@ -44,6 +43,12 @@ MUTANTS = {
     "copy_skips_v": ("            dst_v[dst * per_block + e] = src_v[src * per_block + e];\n", ""),
     "copy_half_block": ("const int64_t per_block = num_kv_heads * block_size * head_dim;",
                         "const int64_t per_block = block_size * head_dim;"),
+    "causal_off_by_one": ("K, V, pos + 1, head_dim", "K, V, pos, head_dim"),
+    "causal_sees_future": ("K, V, pos + 1, head_dim", "K, V, L, head_dim"),
+    "position_top_left": ("int64_t pos = L - n + t;", "int64_t pos = t;"),
+    "prefill_token_row": ("int64_t tok = query_start[s] + t;", "int64_t tok = t;"),
+    "prefill_interleaved_groups": ("for (int64_t hq = h * group; hq < (h + 1) * group; ++hq)",
+                                   "for (int64_t hq = h; hq < num_q_heads; hq += num_kv_heads)"),
     "zero_length_garbage": ("for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;\n            if (L == 0) continue;",
                             "if (L == 0) { o[0] = 1.0; continue; }\n            for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;"),
 }
