@@ -15,6 +15,7 @@
 #include <cudaTypedefs.h>
 
 #include "pa_b200.h"
+#include "pa_copy.cuh"
 #include "pa_kernels.cuh"
 #include "pa_mma.cuh"
 
@@ -628,8 +629,8 @@ int pa_swap_blocks(const void *src_k, const void *src_v, void *dst_k, void *dst_
   a.chunks_per_block = (long long)num_kv_heads * block_size * head_dim * 2 / 16;
   a.src_blocks = src_num_blocks;
   a.dst_blocks = dst_num_blocks;
-  const long long work = num_pairs * 2 * ((a.chunks_per_block + 3) / 4);
-  const int grid = (int)std::max(1LL, std::min<long long>((work + 255) / 256, (long long)sms * 8));
+  const long long warp_tiles = num_pairs * 2 * ((a.chunks_per_block + pa::COPY_TILE - 1) / pa::COPY_TILE);
+  const int grid = (int)std::max(1LL, std::min<long long>((warp_tiles + 7) / 8, (long long)sms * 8));
   cudaError_t e = launch_pdl(pa::copy_blocks_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), a);
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);

@@ -118,55 +118,6 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const WriteArgs a) {
   }
 }
 
-// ---------------------------------------------------------------- block copy
-struct CopyArgs {
-  const uint4 *src_k;
-  const uint4 *src_v;
-  uint4 *dst_k;
-  uint4 *dst_v;
-  const int64_t *mapping;  // [num_pairs][2] (source block, destination block)
-  long long num_pairs, chunks_per_block, src_blocks, dst_blocks;
-};
-
-// Copies whole blocks, K then V, 16 bytes per element of work; each thread
-// moves 4 chunks of one block at a time with the loads issued before the
-// stores.  A pair with a negative entry is skipped; one outside its pool is
-// skipped and flagged.  Either pool may be pinned host memory (unified
-// addressing), which makes the same kernel the swap path.
-__global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyArgs a) {
-  grid_dependency_wait();
-  grid_launch_dependents();
-  constexpr int U = 4;
-  const long long groups = (a.chunks_per_block + U - 1) / U;  // per block and cache
-  const long long total = a.num_pairs * 2 * groups;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long pair = i / (2 * groups);
-    const long long rem = i - pair * 2 * groups;
-    const bool is_v = rem >= groups;
-    const long long g = is_v ? rem - groups : rem;
-    const long long src = a.mapping[2 * pair], dst = a.mapping[2 * pair + 1];  // may be host memory
-    if (src < 0 || dst < 0) continue;
-    if (src >= a.src_blocks || dst >= a.dst_blocks) {
-      if (g == 0 && !is_v) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
-      continue;
-    }
-    const uint4 *from = (is_v ? a.src_v : a.src_k) + src * a.chunks_per_block;
-    uint4 *to = (is_v ? a.dst_v : a.dst_k) + dst * a.chunks_per_block;
-    uint4 v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long c = g * U + u;
-      if (c < a.chunks_per_block) v[u] = from[c];
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long c = g * U + u;
-      if (c < a.chunks_per_block) to[c] = v[u];
-    }
-  }
-}
-
 // ---------------------------------------------------------------- K2/K3: decode
 //
 // Work decomposition ("split over a tile stream"): every sequence s with a
