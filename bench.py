@@ -51,8 +51,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.NAMED))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--op", default="decode", choices=["decode"] + sorted(BLOCK_OPS),
-                    help="decode step (default) or one of the block operations")
+    ap.add_argument("--op", default="decode", choices=["decode", "prefill"] + sorted(BLOCK_OPS),
+                    help="decode step (default), paged prefill, or one of the block operations")
+    ap.add_argument("--prefill-workload", default="llama2_7b_prefill", choices=sorted(W.PREFILL_NAMED))
     ap.add_argument("--pairs", type=int, default=None, help="block pairs per step (block operations)")
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -430,10 +431,161 @@ def run_block_op(args):
     return 0
 
 
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst; fp16 has the same nominal rate)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def oracle_prefill_rate(case, seconds: float):
+    """The oracle on the shortest sequences of the case, one after another, until `seconds` pass."""
+    import oracle
+    qs, lens = case.query_start, case.context_lens
+    order = np.argsort(lens)
+    flops, done, t0 = 0, 0, time.perf_counter()
+    for s in order:
+        s = int(s)
+        n = int(qs[s + 1] - qs[s])
+        L = int(lens[s])
+        oracle.prefill(case.q[qs[s]:qs[s + 1]], case.k_cache, case.v_cache, case.block_tables[s:s + 1],
+                       np.array([0, n], np.int32), lens[s:s + 1], case.scale, case.dtype)
+        flops += 4 * case.head_dim * case.num_q_heads * (n * (L - n) + n * (n + 1) // 2)
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    secs = time.perf_counter() - t0
+    return flops / secs / 1e12, f"{done} of {case.num_seqs} sequences (shortest first), {secs:.1f} s, single thread"
+
+
+def run_prefill_op(args):
+    """Times pa_prefill on a named prefill configuration; prints one JSON line."""
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_457_b200 as pa
+
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+    pa.load_library()
+    case = W.PREFILL_NAMED[args.prefill_workload](seed=6 + 100 * rank if args.prefill_workload == "llama2_7b_prefill"
+                                                  else 7 + 100 * rank)
+    tdt = torch.float16 if case.dtype == "fp16" else torch.bfloat16
+
+    def dev_bits(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(tdt)
+
+    kc, vc, q = dev_bits(case.k_cache), dev_bits(case.v_cache), dev_bits(case.q)
+    tables = torch.from_numpy(case.block_tables).to(device)
+    qs = torch.from_numpy(case.query_start).to(device)
+    lens = torch.from_numpy(case.context_lens).to(device)
+    out = torch.empty_like(q)
+    mql = case.max_query_len
+    flops = 4 * case.head_dim * case.num_q_heads * case.attended_pairs
+
+    def step(qq=q, ss=qs, ll=lens, tt=tables):
+        pa.prefill(qq, kc, vc, tt, ss, ll, case.scale, mql, out=out)
+
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device).start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = pa.launch_count()
+    wall0 = time.perf_counter()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    launches = pa.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    status = pa.device_status()
+
+    # end to end: q and the batch metadata from pinned host memory, the output back to pinned host memory
+    hq_ = torch.from_numpy(case.q.view(np.int16)).pin_memory()
+    hmeta = [torch.from_numpy(a).pin_memory() for a in (case.query_start, case.context_lens, case.block_tables)]
+    out_host = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+    dq = torch.empty_like(q)
+    dqs, dlens, dtables = torch.empty_like(qs), torch.empty_like(lens), torch.empty_like(tables)
+
+    def e2e_step():
+        dq.view(torch.int16).copy_(hq_, non_blocking=True)
+        dqs.copy_(hmeta[0], non_blocking=True)
+        dlens.copy_(hmeta[1], non_blocking=True)
+        dtables.copy_(hmeta[2], non_blocking=True)
+        step(dq, dqs, dlens, dtables)
+        out_host.copy_(out.view(torch.int16), non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / args.steps
+    h2d = hq_.numel() * 2 + sum(t.numel() * t.element_size() for t in hmeta)
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, sample = oracle_prefill_rate(case, min(args.cpu_sample_seconds, 10.0))
+        cpu = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample}
+    if rank == 0:
+        peak, peak_kind = measured_tensor_peak()
+        achieved = flops / (ms / 1e3) / 1e12
+        line = {
+            "metric": "paged causal prefill attention TFLOP/s (fraction of tensor peak), 1×B200",
+            "value": round(world * achieved, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": case.dtype, "data": "synthetic",
+            "tokens_per_s": round(world * int(case.query_start[-1]) / (ms / 1e3), 1),
+            "config": {"workload": case.name, "description": case.description, "num_seqs": case.num_seqs,
+                       "new_tokens": int(case.query_start[-1]), "attended_pairs": case.attended_pairs,
+                       "num_q_heads": case.num_q_heads, "num_kv_heads": case.num_kv_heads,
+                       "head_dim": case.head_dim, "block_size": case.block_size,
+                       "parallelism": f"dp{world} (independent batches per GPU)",
+                       "l2": "no flush: K/V of the batch exceed the 126 MB L2"},
+            "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 1),
+                         "peak": peak, "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "traffic": None, "algorithmic_flops": flops, "ms_per_launch": round(ms, 5)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(world * flops / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_host.numel() * 2),
+                    "ms_per_step": round(e2e_ms, 4)},
+            "gpu_launches": int(launches), "clocks": sampler.summary(wall0, wall1), "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "prefill":
+        return run_prefill_op(args)
     if args.op != "decode":
         return run_block_op(args)
 

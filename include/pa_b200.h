@@ -155,6 +155,40 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
               int32_t partition_tokens, int32_t dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * pa_prefill -- causal attention of each sequence's NEW tokens (a prompt, or
+ * the next chunk of one) over its paged context ("4. vLLM核心机制" section
+ * 4.3: the prompt's tokens enter the cache before decoding starts, possibly
+ * a piece per iteration).  Sequence s brings
+ * n_s = query_start[s+1] - query_start[s] new tokens whose K/V rows are
+ * ALREADY in the cache (write them with pa_write_kv first); its context
+ * holds L_s = context_lens[s] >= n_s tokens, the new ones last.  New token t
+ * (0 <= t < n_s) is at logical position p = L_s - n_s + t and attends to the
+ * tokens 0..p only:
+ *   out[query_start[s] + t][hq][:] = softmax_j(scale * q . K[j]) V[j],  j = 0..p,
+ * K/V rows gathered through block_tables as in pa_decode (kv head
+ * hq / (num_q_heads / num_kv_heads)).  n_s = 1 is a decode step.
+ *   q            [num_query_tokens][num_q_heads][head_dim], token stride
+ *                q_token_stride (elements, multiple of 8);
+ *   query_start  int32 [num_seqs + 1], query_start[0] = 0, non-decreasing,
+ *                query_start[num_seqs] <= num_query_tokens;
+ *   context_lens int32 [num_seqs];
+ *   out          like q, token stride out_token_stride;
+ *   max_query_len >= every n_s (sizes the grid; rows past it are not computed).
+ * Runs on the tensor cores (tcgen05, tensor memory accumulators), 128 new
+ * tokens of one query head per CTA; computes in fp32 with P rounded to the
+ * storage type.  Device-side errors: L_s < n_s or L_s > block_table_stride *
+ * block_size -> PA_DEV_ERR_CONTEXT and zero rows; query_start entries that
+ * leave [0, num_query_tokens] -> PA_DEV_ERR_CONTEXT and that sequence is not
+ * written; a needed table entry outside the pool -> PA_DEV_ERR_BLOCK_ID and
+ * zero rows.
+ */
+int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+               const int32_t *query_start, const int32_t *context_lens, float scale, void *out, int32_t num_seqs,
+               int64_t num_query_tokens, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+               int32_t block_size, int64_t num_blocks, int32_t block_table_stride, int32_t max_query_len,
+               int64_t q_token_stride, int64_t out_token_stride, int32_t dtype, void *stream);
+
+/*
  * pa_copy_blocks -- copy whole blocks inside one pair of caches: for every
  * pair i, block block_mapping[i][0] is copied (all kv heads, rows and dims, K
  * and V) to block block_mapping[i][1].  This is the copy a sequence needs

@@ -24,7 +24,7 @@ import threading
 import torch
 
 __all__ = [
-    "PagedAttentionError", "write_kv", "decode", "decode_workspace_size", "copy_blocks", "swap_blocks",
+    "PagedAttentionError", "write_kv", "decode", "decode_workspace_size", "copy_blocks", "swap_blocks", "prefill",
     "device_status", "launch_count", "debug_wait_timeout", "library_path", "load_library", "EXPORTED_SYMBOLS",
     "DEV_ERR_BLOCK_ID", "DEV_ERR_CONTEXT", "DEV_ERR_CONTEXT_HINT", "DEV_ERR_SLOT", "DEV_ERR_TIMEOUT",
     "BlockManager", "BlockManagerError", "DecodeStepPlan",
@@ -50,7 +50,7 @@ EXPORTED_SYMBOLS = (
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_device_blocks", "pa_bm_num_free_host_blocks",
     "pa_bm_ref_count", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_num_tokens",
     "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step",
-    "pa_bm_swap_out", "pa_bm_swap_in",
+    "pa_bm_swap_out", "pa_bm_swap_in", "pa_prefill",
 )
 
 
@@ -98,6 +98,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_copy_blocks.argtypes = [vp, vp, vp, i64, i32, i32, i32, i64, vp]
         lib.pa_swap_blocks.restype = ctypes.c_int
         lib.pa_swap_blocks.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, i64, vp]
+        lib.pa_prefill.restype = ctypes.c_int
+        lib.pa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, f32, vp, i32, i64, i32, i32, i32, i32, i64, i32, i32, i64,
+                                   i64, i32, vp]
         lib.pa_version.restype = i32
         lib.pa_version.argtypes = []
         from .block_manager import bind as _bind_block_manager
@@ -221,6 +224,43 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
                        workspace.data_ptr() if workspace is not None else None,
                        workspace.numel() * workspace.element_size() if workspace is not None else 0, stream)
     _check(rc, "pa_decode")
+    return out
+
+
+def prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+            query_start: torch.Tensor, context_lens: torch.Tensor, scale: float, max_query_len: int,
+            out: torch.Tensor | None = None) -> torch.Tensor:
+    """Causal attention of each sequence's new tokens over its paged context (K/V already written).
+
+    q: [N, Hq, d] (token rows of all sequences, back to back); query_start: int32 [S + 1];
+    context_lens: int32 [S] (new tokens included); max_query_len >= every sequence's new tokens.
+    """
+    dev = k_cache.device
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("block_tables", block_tables),
+                    ("query_start", query_start), ("context_lens", context_lens)):
+        _need_cuda(name, t, dev)
+    nb, hkv, bs, d = _cache_geometry(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != d or q.dtype != k_cache.dtype or q.stride(2) != 1 or q.stride(1) != d:
+        raise PagedAttentionError("q must be [N, Hq, head_dim] with contiguous heads, same dtype as the caches")
+    S = int(context_lens.shape[0])
+    for name, t, shape in (("query_start", query_start, (S + 1,)), ("context_lens", context_lens, (S,))):
+        if t.dtype != torch.int32 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise PagedAttentionError(f"{name} must be a contiguous int32 tensor of shape {shape}")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != S \
+            or block_tables.stride(1) != 1:
+        raise PagedAttentionError("block_tables must be int32 [S, max_blocks] with unit column stride")
+    N, hq = int(q.shape[0]), int(q.shape[1])
+    if out is None:
+        out = torch.empty((N, hq, d), dtype=q.dtype, device=dev)
+    else:
+        _need_cuda("out", out, dev)
+        if tuple(out.shape) != (N, hq, d) or out.dtype != q.dtype or out.stride(2) != 1 or out.stride(1) != d:
+            raise PagedAttentionError("out must match q's shape and dtype, heads contiguous")
+    rc = load_library().pa_prefill(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
+                                   query_start.data_ptr(), context_lens.data_ptr(), float(scale), out.data_ptr(), S, N,
+                                   hq, hkv, d, bs, nb, int(block_tables.stride(0)), int(max_query_len),
+                                   int(q.stride(0)), int(out.stride(0)), _DTYPES[k_cache.dtype], _stream(dev))
+    _check(rc, "pa_prefill")
     return out
 
 

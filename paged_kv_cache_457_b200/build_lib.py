@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpa_b200.so")
 SOURCES = [os.path.join(CSRC, "pa_api.cu"), os.path.join(CSRC, "block_manager.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_mma.cuh", "pa_ptx.cuh", "pa_copy.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_mma.cuh", "pa_ptx.cuh", "pa_copy.cuh", "pa_prefill.cuh", "pa_tcgen05.cuh")] + [
     os.path.join(INCLUDE, h) for h in ("pa_b200.h", "pa_block_manager.h")]
 
 

@@ -17,6 +17,7 @@
 #include "pa_b200.h"
 #include "pa_copy.cuh"
 #include "pa_kernels.cuh"
+#include "pa_prefill.cuh"
 #include "pa_mma.cuh"
 
 namespace {
@@ -641,6 +642,92 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int64_t num_blocks, void *stream) {
   return pa_swap_blocks(k_cache, v_cache, k_cache, v_cache, block_mapping, num_pairs, num_kv_heads, head_dim,
                         block_size, num_blocks, num_blocks, stream);
+}
+
+int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+               const int32_t *query_start, const int32_t *context_lens, float scale, void *out, int32_t num_seqs,
+               int64_t num_query_tokens, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+               int32_t block_size, int64_t num_blocks, int32_t block_table_stride, int32_t max_query_len,
+               int64_t q_token_stride, int64_t out_token_stride, int32_t dtype, void *stream) {
+  if (num_seqs < 0 || num_query_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_query_len < 0 ||
+      num_blocks < 0 || block_table_stride < 0)
+    return PA_ERR_SHAPE;
+  if (num_seqs > 65535 || num_q_heads > 65535 || num_query_tokens > 0x7fffffffLL) return PA_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_HEADS;
+  if (dtype != PA_FLOAT16 && dtype != PA_BFLOAT16) return PA_ERR_DTYPE;
+  if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if (num_seqs == 0 || num_query_tokens == 0 || max_query_len == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !query_start || !context_lens || !out) return PA_ERR_NULL;
+  if (q_token_stride < (long long)num_q_heads * head_dim || out_token_stride < (long long)num_q_heads * head_dim)
+    return PA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || (q_token_stride % 8) ||
+      (out_token_stride % 8))
+    return PA_ERR_ALIGN;
+  const long long rows = num_blocks * num_kv_heads * block_size;
+  if (rows > 0x7fffffffLL || rows == 0) return PA_ERR_SHAPE;  // TMA coordinates are signed 32-bit
+  int rc = PA_OK;
+  auto encode = tensor_map_encoder(&rc);
+  if (!encode) return rc;
+  CUtensorMap mq, mk, mv;
+  {
+    // q viewed as [tokens][heads][head_dim]; one box = 128 tokens x 64 dims of one head
+    const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads, (cuuint64_t)num_query_tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)q_token_stride * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)pa::PF_BM};
+    const cuuint32_t elem_strides[3] = {1, 1, 1};
+    const CUresult r =
+        encode(&mq, dtype == PA_BFLOAT16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+               const_cast<void *>(q), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      t_last_cuda_error = "cuTensorMapEncodeTiled failed for q (code " + std::to_string((int)r) + ")";
+      return PA_ERR_CUDA;
+    }
+  }
+  rc = cache_tensor_map(k_cache, rows, head_dim, dtype, &mk);
+  if (rc != PA_OK) return rc;
+  rc = cache_tensor_map(v_cache, rows, head_dim, dtype, &mv);
+  if (rc != PA_OK) return rc;
+
+  pa::PrefillArgs a;
+  a.block_tables = block_tables;
+  a.query_start = query_start;
+  a.context_lens = context_lens;
+  a.out = static_cast<uint16_t *>(out);
+  a.num_blocks = num_blocks;
+  a.out_token_stride = out_token_stride;
+  a.num_query_tokens = num_query_tokens;
+  a.wait_limit_ns = kWaitLimitNs;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);  // log2(e)
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.block_size = block_size;
+  a.table_stride = block_table_stride;
+  a.q_tiles = (max_query_len + pa::PF_BM - 1) / pa::PF_BM;
+  const dim3 grid(a.q_tiles, num_q_heads, num_seqs);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto launch = [&](auto kernel, uint32_t smem) -> int {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return record(e);
+    e = launch_pdl(kernel, grid, dim3(pa::PF_THREADS), smem, st, mq, mk, mv, a);
+    if (e != cudaSuccess) return record(e);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return record(e);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PA_OK;
+  };
+  constexpr int kPrefillStages = 2;
+  if (dtype == PA_BFLOAT16) {
+    if (head_dim == 128)
+      return launch(pa::prefill_tc_kernel<pa::BF16, 128, kPrefillStages>, pa::PrefillSmem<128, kPrefillStages>::ALLOC);
+    return launch(pa::prefill_tc_kernel<pa::BF16, 64, kPrefillStages>, pa::PrefillSmem<64, kPrefillStages>::ALLOC);
+  }
+  if (head_dim == 128)
+    return launch(pa::prefill_tc_kernel<pa::F16, 128, kPrefillStages>, pa::PrefillSmem<128, kPrefillStages>::ALLOC);
+  return launch(pa::prefill_tc_kernel<pa::F16, 64, kPrefillStages>, pa::PrefillSmem<64, kPrefillStages>::ALLOC);
 }
 
 int32_t pa_version(void) { return 100; }

@@ -338,6 +338,113 @@ def shared_prefix(seed: int = 5, num_steps: int = 16, groups: int = 8, seqs_per_
                                 f"group 0 retires after step {retire_after}")
 
 
+@dataclass
+class PrefillCase:
+    """Causal prefill of new tokens over a paged context whose K/V rows (the new tokens' included)
+    are already in the pool: sequence s brings query rows query_start[s]..query_start[s+1]-1, the
+    last n_s of its context_lens[s] tokens."""
+
+    name: str
+    dtype: str
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    scale: float
+    k_cache: np.ndarray  # uint16 [NB, Hkv, bs, d]
+    v_cache: np.ndarray
+    q: np.ndarray  # uint16 [N, Hq, d]
+    query_start: np.ndarray  # int32 [S + 1]
+    context_lens: np.ndarray  # int32 [S]
+    block_tables: np.ndarray  # int32 [S, MB]
+    description: str = ""
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.context_lens.shape[0])
+
+    @property
+    def query_lens(self) -> np.ndarray:
+        return np.diff(self.query_start)
+
+    @property
+    def max_query_len(self) -> int:
+        return int(self.query_lens.max(initial=0))
+
+    @property
+    def attended_pairs(self) -> int:
+        """Sum over new tokens of the keys each attends to (causal)."""
+        total = 0
+        for L, n in zip(self.context_lens.astype(np.int64), self.query_lens.astype(np.int64)):
+            total += int(n * (L - n) + n * (n + 1) // 2)
+        return total
+
+
+def prefill_case(seed: int, shape, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
+                 dtype: str = "fp16", num_blocks: int | None = None, table_width: int | None = None,
+                 name: str = "custom_prefill", description: str = "") -> PrefillCase:
+    """shape: [(L, n)] per sequence (context length, new tokens).  Blocks come from a shuffled free
+    list; unowned slots hold NaN."""
+    draw = _Draw(seed)
+    lens = [int(L) for L, _ in shape]
+    ns = [int(n) for _, n in shape]
+    assert all(0 <= n <= L for L, n in zip(lens, ns))
+    bs = block_size
+    need = sum(-(-L // bs) for L in lens)
+    nb = num_blocks if num_blocks is not None else need + 3
+    if need > nb:
+        raise ValueError(f"{name}: pool of {nb} blocks too small for {need}")
+    width = table_width if table_width is not None else max(1, max((-(-L // bs) for L in lens), default=1))
+    free = draw.np.permutation(nb).astype(np.int32)
+    k_cache = _nan_pool(nb, num_kv_heads, bs, head_dim, dtype)
+    v_cache = _nan_pool(nb, num_kv_heads, bs, head_dim, dtype)
+    tables = np.full((len(lens), width), TABLE_PAD, dtype=np.int32)
+    cursor = 0
+    for s, L in enumerate(lens):
+        nblk = -(-L // bs)
+        tables[s, :nblk] = free[cursor:cursor + nblk]
+        cursor += nblk
+        for t0 in range(0, L, 8192):
+            t1 = min(L, t0 + 8192)
+            _place(k_cache, tables[s], t0, draw.normal_bits((t1 - t0, num_kv_heads, head_dim), dtype), bs)
+            _place(v_cache, tables[s], t0, draw.normal_bits((t1 - t0, num_kv_heads, head_dim), dtype), bs)
+    qs = np.concatenate([[0], np.cumsum(ns)]).astype(np.int32)
+    q = draw.normal_bits((int(qs[-1]), num_q_heads, head_dim), dtype)
+    return PrefillCase(name=name, dtype=dtype, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+                       head_dim=head_dim, block_size=bs, num_blocks=nb, scale=1.0 / math.sqrt(head_dim),
+                       k_cache=k_cache, v_cache=v_cache, q=q, query_start=qs,
+                       context_lens=np.asarray(lens, dtype=np.int32), block_tables=tables, description=description)
+
+
+def prefill_llama2_7b(seed: int = 6, num_seqs: int = 16, num_blocks: int = 4096) -> PrefillCase:
+    """Llama-2-7B-shaped prompt prefill: 16 prompts of U{512..2048} tokens, 32 heads, d=128, bs=16,
+    fp16, whole prompt in one pass; 4096-block shuffled pool."""
+    rng = np.random.Generator(np.random.PCG64(seed + 1000))
+    lens = rng.integers(512, 2049, size=num_seqs)
+    return prefill_case(seed, [(int(L), int(L)) for L in lens], 32, 32, 128, 16, "fp16", num_blocks, 128,
+                        name="llama2_7b_prefill",
+                        description=f"{num_seqs} prompts, L~U[512,2048], 32 heads, d128, bs16, fp16, "
+                                    f"{num_blocks}-block pool")
+
+
+def chunked_prefill_gqa(seed: int = 7, num_seqs: int = 32, chunk: int = 512, num_blocks: int = 16384) -> PrefillCase:
+    """Chunked prefill, GQA 32 q / 8 kv heads, d=128, bs=16, bf16: each sequence has a cached prefix
+    of U{0..3584} tokens and brings the next chunk of 512; 16384-block pool."""
+    rng = np.random.Generator(np.random.PCG64(seed + 1000))
+    prefix = rng.integers(0, 3585, size=num_seqs)
+    return prefill_case(seed, [(int(p) + chunk, chunk) for p in prefix], 32, 8, 128, 16, "bf16", num_blocks, 256,
+                        name="gqa_chunked_prefill",
+                        description=f"{num_seqs} seqs, cached prefix U[0,3584] + chunk {chunk}, 32q/8kv heads, "
+                                    f"d128, bs16, bf16, {num_blocks}-block pool")
+
+
+PREFILL_NAMED = {
+    "llama2_7b_prefill": prefill_llama2_7b,
+    "gqa_chunked_prefill": chunked_prefill_gqa,
+}
+
+
 NAMED = {
     "tiny_decode": tiny,
     "llama2_7b_decode": llama2_7b,
