@@ -707,7 +707,12 @@ int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const in
   a.block_size = block_size;
   a.table_stride = block_table_stride;
   a.q_tiles = (max_query_len + pa::PF_BM - 1) / pa::PF_BM;
-  const dim3 grid(a.q_tiles, num_q_heads, num_seqs);
+  a.num_items = (long long)a.q_tiles * num_q_heads * num_seqs;
+  int sms = 0;
+  rc = current_sms(&sms);
+  if (rc != PA_OK) return rc;
+  // persistent: one CTA per SM (the shared-memory footprint admits no second one)
+  const dim3 grid((unsigned)std::min<long long>(a.num_items, sms));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto launch = [&](auto kernel, uint32_t smem) -> int {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -719,15 +724,12 @@ int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const in
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return PA_OK;
   };
-  constexpr int kPrefillStages = 2;
   if (dtype == PA_BFLOAT16) {
-    if (head_dim == 128)
-      return launch(pa::prefill_tc_kernel<pa::BF16, 128, kPrefillStages>, pa::PrefillSmem<128, kPrefillStages>::ALLOC);
-    return launch(pa::prefill_tc_kernel<pa::BF16, 64, kPrefillStages>, pa::PrefillSmem<64, kPrefillStages>::ALLOC);
+    if (head_dim == 128) return launch(pa::prefill_tc_kernel<pa::BF16, 128>, pa::PrefillSmem<128>::ALLOC);
+    return launch(pa::prefill_tc_kernel<pa::BF16, 64>, pa::PrefillSmem<64>::ALLOC);
   }
-  if (head_dim == 128)
-    return launch(pa::prefill_tc_kernel<pa::F16, 128, kPrefillStages>, pa::PrefillSmem<128, kPrefillStages>::ALLOC);
-  return launch(pa::prefill_tc_kernel<pa::F16, 64, kPrefillStages>, pa::PrefillSmem<64, kPrefillStages>::ALLOC);
+  if (head_dim == 128) return launch(pa::prefill_tc_kernel<pa::F16, 128>, pa::PrefillSmem<128>::ALLOC);
+  return launch(pa::prefill_tc_kernel<pa::F16, 64>, pa::PrefillSmem<64>::ALLOC);
 }
 
 int32_t pa_version(void) { return 100; }
