@@ -706,7 +706,7 @@ int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const in
   a.num_kv_heads = num_kv_heads;
   a.block_size = block_size;
   a.table_stride = block_table_stride;
-  a.q_tiles = (max_query_len + pa::PF_BM - 1) / pa::PF_BM;
+  a.q_tiles = (max_query_len + pa::PF_ROWS - 1) / pa::PF_ROWS;
   a.num_items = (long long)a.q_tiles * num_q_heads * num_seqs;
   int sms = 0;
   rc = current_sms(&sms);

@@ -2,26 +2,30 @@
 // sm_100a tensor cores ("4. vLLM核心机制" section 4.3: the prompt's tokens
 // enter the cache before decoding, possibly a chunk per iteration).
 //
-// Work item: 128 consecutive new tokens of one sequence for one query head.
-// Persistent CTAs (one per SM) walk the items round-robin; the items of one
-// (sequence, head) are adjacent, so the CTAs working on them at the same time
-// share that head's K/V through L2, and the latest (heaviest) query tiles of
-// a sequence come first.  Per key tile of 128 tokens (8 pages of 16 or 4 of 32):
-//   S = Q K^T      tcgen05.mma M=128 N=128 K=d, Q and K tiles in swizzled smem,
-//                  S in tensor memory (two buffers, so the next tile's S is
-//                  computed while this one's softmax runs);
-//   softmax        4 warps, one row each: S read from tensor memory, causal
-//                  mask, online max with a lazy rescale of O, P rounded to the
-//                  storage type and written to smem in the MMA's swizzled layout;
-//   O += P V       tcgen05.mma M=128 N=d K=128, V read MN-major straight from
-//                  its TMA tile, O accumulated in tensor memory.
-// Warp roles: 0-3 softmax and epilogue, 4 TMA producer of Q (two buffers) and
-// K pages, 5 MMA issue (one lane), 6 TMA producer of V pages.  A K slot frees
-// when its QK^T has run, a V slot when its PV has, so K runs ahead of V.  The
-// MMA lane keeps one software pipeline across items: QK^T of tile g, then PV
-// of tile g-1.  Every wait is bounded: on a timeout the CTA flags
-// PA_DEV_ERR_TIMEOUT, drains its copies and MMAs in flight, frees its tensor
-// memory and returns.
+// Work item: 256 consecutive new tokens of one sequence for one query head,
+// as two 128-row sub-tiles A and B that share every K/V tile (half the K/V
+// bytes per flop of one 128-row tile).  Persistent CTAs (one per SM) walk the
+// items round-robin; the items of one (sequence, head) are adjacent, so the
+// CTAs working on them at the same time share that head's K/V through L2, and
+// the latest (heaviest) query tiles come first.  Per key tile of 128 tokens
+// (8 pages of 16 or 4 of 32), for each sub-tile x:
+//   S_x = Q_x K^T    tcgen05.mma M=128 N=128 K=d, Q and K from swizzled smem,
+//                    S_x in tensor memory;
+//   softmax_x        one warpgroup per sub-tile, one row per thread: S_x read
+//                    from tensor memory (twice: max, then exponentials),
+//                    causal mask, online max with a lazy rescale of O_x, P_x
+//                    rounded to the storage type and stored back into the
+//                    first half of S_x's columns;
+//   O_x += P_x V     tcgen05.mma M=128 N=d K=128 with P_x read from tensor
+//                    memory and V MN-major from its TMA tile.
+// The MMA lane issues QK_A(j), PV_B(j-1), QK_B(j), PV_A(j): each warpgroup's
+// softmax runs while the tensor core works on the other sub-tile.  Tensor
+// memory (512 columns): S_A, S_B (128 each), O_A, O_B (d each).
+// Warp roles: 0-3 softmax of A, 4-7 softmax of B, 8 TMA producer of Q and K
+// pages, 9 TMA producer of V pages, 10 MMA issue (one lane).  A K slot frees
+// once both QK^T of its tile ran, a V slot once both PV did.  Every wait is
+// bounded: on a timeout the CTA flags PA_DEV_ERR_TIMEOUT, drains its copies
+// and MMAs in flight, frees its tensor memory and returns.
 #pragma once
 
 #include <cuda.h>
@@ -45,25 +49,28 @@ struct PrefillArgs {
   int num_seqs, num_q_heads, num_kv_heads, block_size, table_stride, q_tiles;
 };
 
-constexpr int PF_BM = 128;  // query rows per item
-constexpr int PF_BN = 128;  // keys per tile
-constexpr int PF_THREADS = 224;
-constexpr int PF_KST = 2;  // K ring
-constexpr int PF_VST = 2;  // V ring
-constexpr uint32_t PF_TMEM_COLS = 512;  // S double buffer (2 x 128) + O (<= 128), rounded to a power of two
+constexpr int PF_BM = 128;             // query rows per sub-tile
+constexpr int PF_ROWS = 2 * PF_BM;     // query rows per item (sub-tiles A and B)
+constexpr int PF_BN = 128;             // keys per tile
+constexpr int PF_THREADS = 11 * 32;
+constexpr int PF_KST = 3;              // K ring
+constexpr int PF_VST = 2;              // V ring
+constexpr uint32_t PF_TMEM_COLS = 512;
 
 template <int D>
 struct PrefillSmem {
   static constexpr uint32_t REGION = 128 * 128;  // 128 rows of 128 bytes (64 elements)
   static constexpr uint32_t HALVES = D / 64;
-  static constexpr uint32_t Q = 0;  // two buffers
+  static constexpr uint32_t Q = 0;  // sub-tiles A and B
   static constexpr uint32_t K = Q + 2 * HALVES * REGION;
   static constexpr uint32_t V = K + PF_KST * HALVES * REGION;
-  static constexpr uint32_t P = V + PF_VST * HALVES * REGION;
-  static constexpr uint32_t BARS = P + 2 * REGION;
+  static constexpr uint32_t BARS = V + PF_VST * HALVES * REGION;
   static constexpr uint32_t BYTES = BARS + 256;
   // + alignment slack; at least 120 KB so that one CTA holds an SM (and its tensor memory) alone
   static constexpr uint32_t ALLOC = (BYTES + 1024 > 120 * 1024) ? BYTES + 1024 : 120 * 1024;
+  // tensor memory columns
+  static constexpr uint32_t T_S = 0;      // S_x at T_S + x * 128; P_x in its first 64 columns
+  static constexpr uint32_t T_O = 256;    // O_x at T_O + x * D
 };
 
 // 2^x with the SFU's approximate exponential (documented PTX; relative error about 2^-22, 2^-inf = 0).
@@ -81,8 +88,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
 
 // One work item as every role sees it (all values uniform across the CTA).
 struct PrefillItem {
-  int s, hq, h, q0, t0, rows, ctx, pos0, kmax, nt;
-  bool work, bad_ctx;
+  int s, hq, h, q0, t0, rows, ctx, pos0, kmax, nt, nt_a;
+  bool work, bad_ctx, has_b;
 };
 
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillArgs &a, long long item) {
@@ -96,24 +103,26 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillArgs &a, long l
   it.q0 = a.query_start[it.s];
   const int n = a.query_start[it.s + 1] - it.q0;
   it.ctx = a.context_lens[it.s];
-  it.t0 = qt * PF_BM;
-  it.work = false;
-  it.bad_ctx = false;
-  it.rows = it.pos0 = it.kmax = it.nt = 0;
+  it.t0 = qt * PF_ROWS;
+  it.work = it.bad_ctx = it.has_b = false;
+  it.rows = it.pos0 = it.kmax = it.nt = it.nt_a = 0;
   if (it.q0 < 0 || n < 0 || (long long)it.q0 + n > a.num_query_tokens) {  // rows outside q / out
     if (qt == a.q_tiles - 1 && it.hq == 0 && threadIdx.x == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
     return it;
   }
   if (it.t0 >= n) return it;
-  it.rows = min(PF_BM, n - it.t0);
+  it.rows = min(PF_ROWS, n - it.t0);
   if (it.ctx < n || (long long)it.ctx > (long long)a.table_stride * a.block_size) {
     it.bad_ctx = true;
     return it;
   }
   it.work = true;
-  it.pos0 = it.ctx - n + it.t0;              // logical position of row 0
+  it.has_b = it.rows > PF_BM;
+  it.pos0 = it.ctx - n + it.t0;              // logical position of row 0 of sub-tile A
   it.kmax = min(it.ctx, it.pos0 + it.rows);  // keys [0, kmax) are visible to some row
   it.nt = (it.kmax + PF_BN - 1) / PF_BN;
+  // sub-tile A sees keys up to pos0 + 127 only; its tiles are a prefix of the item's
+  it.nt_a = (min(it.kmax, it.pos0 + PF_BM) + PF_BN - 1) / PF_BN;
   return it;
 }
 
@@ -171,27 +180,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   uint8_t *sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const uint32_t sbase = smem_addr(sm);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BARS);
-  uint64_t *q_full = bars;              // [2]
-  uint64_t *q_empty = q_full + 2;       // [2]
-  uint64_t *k_full = q_empty + 2;       // [PF_KST]
+  uint64_t *q_full = bars;
+  uint64_t *q_empty = q_full + 1;
+  uint64_t *k_full = q_empty + 1;       // [PF_KST]
   uint64_t *k_empty = k_full + PF_KST;  // [PF_KST]
   uint64_t *v_full = k_empty + PF_KST;  // [PF_VST]
   uint64_t *v_empty = v_full + PF_VST;  // [PF_VST]
-  uint64_t *s_full = v_empty + PF_VST;  // [2]
-  uint64_t *p_full = s_full + 2;
-  uint64_t *o_done = p_full + 1;
-  uint64_t *drained = o_done + 1;
+  uint64_t *s_full = v_empty + PF_VST;  // [2]: S_A, S_B written (and every earlier MMA done)
+  uint64_t *p_full = s_full + 2;        // [2]: P_A, P_B written
+  uint64_t *o_done = p_full + 2;        // [2]: an item's last PV of A, of B done
+  uint64_t *drained = o_done + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drained + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *bad_pages = abort_flag + 1;  // [4]: per item, a ring of 4
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < PF_KST; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -200,14 +206,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
     mbar_init(drained, 1);
     *abort_flag = 0;
     for (int i = 0; i < 4; ++i) bad_pages[i] = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 10) {
     tc::alloc(tmem_slot, PF_TMEM_COLS);
     tc::relinquish();
   }
@@ -218,9 +227,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   const unsigned long long limit = a.wait_limit_ns;
   const long long first = blockIdx.x, stride = gridDim.x;
 
-  if (warp == 4 || warp == 6) {
-    // ------------------------------------------------------------ TMA producers: Q and K (warp 4), V (warp 6)
-    const bool is_k = warp == 4;
+  if (warp == 8 || warp == 9) {
+    // ------------------------------------------------------------ TMA producers: Q and K (warp 8), V (warp 9)
+    const bool is_k = warp == 8;
     if (lane == 0) {
       prefetch_tensor_map(is_k ? &tmap_k : &tmap_v);
       if (is_k) prefetch_tensor_map(&tmap_q);
@@ -236,21 +245,23 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       const PrefillItem it = prefill_item(a, item);
       if (!it.work) continue;
       if (is_k) {
-        const int qb = n_items & 1;
-        if (n_items >= 2 && !(ok = warp_wait(&q_empty[qb], ((n_items >> 1) - 1) & 1, limit))) break;
+        if (n_items >= 1 && !(ok = warp_wait(q_empty, (uint32_t)((n_items - 1) & 1), limit))) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&q_full[qb], PF_BM * D * 2);
+          mbar_arrive_expect_tx(q_full, 2 * PF_BM * D * 2);
 #pragma unroll
-          for (int hh = 0; hh < HALVES; ++hh)
-            tc::tma_load_3d(sm + L::Q + (qb * HALVES + hh) * REGION, &tmap_q, hh * 64, it.hq, it.q0 + it.t0,
-                            &q_full[qb]);
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int hh = 0; hh < HALVES; ++hh)
+              tc::tma_load_3d(sm + L::Q + (x * HALVES + hh) * REGION, &tmap_q, hh * 64, it.hq,
+                              it.q0 + it.t0 + x * PF_BM, q_full);
         }
       }
+      bool any_bad = false;
       bool bad_next;
       int blk_next = tile_page(a, it, 0, lane, &bad_next);
       for (int j = 0; j < it.nt; ++j, ++g) {
         const int blk = blk_next;
-        const bool bad = bad_next;
+        any_bad = any_bad || bad_next;
         if (j + 1 < it.nt) blk_next = tile_page(a, it, j + 1, lane, &bad_next);  // in flight during the wait
         const int st = (int)(g % nst);
         if (g >= nst && !(ok = warp_wait(&empty[st], (uint32_t)(((g / nst) - 1) & 1), limit))) break;
@@ -258,9 +269,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           ok = false;
           break;
         }
-        if (!is_k && __any_sync(FULL, bad) && lane == 0) {
-          bad_pages[n_items & 3] = 1;  // published by this tile's v_full arrival
-          atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
+        if (!is_k && j == it.nt - 1) {  // published by this tile's v_full arrival
+          const bool bad_item = __any_sync(FULL, any_bad);
+          if (lane == 0) {
+            bad_pages[n_items & 3] = bad_item ? 1 : 0;
+            if (bad_item) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
+          }
         }
         load_tile<HALVES>(a, it, blk, lane, ring + st * HALVES * REGION, is_k ? &tmap_k : &tmap_v, &full[st]);
       }
@@ -275,71 +289,86 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       const long long last = i + ((g - 1 - i) / nst) * nst;
       drained_ok = warp_wait(&full[i], (uint32_t)((last / nst) & 1), limit) && drained_ok;
     }
-    if (is_k)
-      for (int i = 0; i < 2 && i < n_items; ++i) {
-        const int last = i + ((n_items - 1 - i) / 2) * 2;
-        drained_ok = warp_wait(&q_full[i], (uint32_t)((last >> 1) & 1), limit) && drained_ok;
-      }
+    if (is_k && n_items > 0) drained_ok = warp_wait(q_full, (uint32_t)((n_items - 1) & 1), limit) && drained_ok;
     if (!drained_ok && lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
-  } else if (warp == 5) {
+  } else if (warp == 10) {
     // ------------------------------------------------------------ MMA issue (one lane)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = tc::idesc_f16(kBf16, false, PF_BM, PF_BN);
       constexpr uint32_t idesc_pv = tc::idesc_f16(kBf16, true, PF_BM, D);
-      const uint32_t ps = sbase + L::P;
-      long long g = 0;         // tiles whose QK^T has been issued
-      long long pending = -1;  // tile whose PV is due next
-      bool pending_first = false;
+      const uint32_t qs = sbase + L::Q;
+      long long g = 0;           // K/V tiles
+      long long gx[2] = {0, 0};  // tiles of sub-tile A, B
       int n_items = 0;
       bool ok = true;
-      // PV of tile t (O += P V), once its softmax has written P.
-      auto issue_pv = [&](long long t, bool first_of_item) -> bool {
-        if (!mbar_wait_bounded(p_full, (uint32_t)(t & 1), limit)) return false;
+      // S_x = Q_x K(t)^T
+      auto issue_qk = [&](int x, long long t) {
+        const uint32_t ks = sbase + L::K + (uint32_t)(t % PF_KST) * HALVES * REGION;
+        const uint32_t qx = qs + x * HALVES * REGION;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * REGION + (k % 4) * 32;
+          tc::mma_ss(tmem + L::T_S + x * 128, tc::desc_sw128(qx + off, 16, 1024), tc::desc_sw128(ks + off, 16, 1024),
+                     idesc_qk, k > 0);
+        }
+        tc::commit(&s_full[x]);
+      };
+      // O_x += P_x V(t), once softmax_x has written P_x for its tile gx
+      auto issue_pv = [&](int x, long long t, long long tx, bool first_of_item) -> bool {
+        if (!mbar_wait_bounded(&p_full[x], (uint32_t)(tx & 1), limit)) return false;
         const int st = (int)(t % PF_VST);
         if (!mbar_wait_bounded(&v_full[st], (uint32_t)((t / PF_VST) & 1), limit)) return false;
         tc::fence_after_sync();
         const uint32_t vs = sbase + L::V + st * HALVES * REGION;
 #pragma unroll
-        for (int k = 0; k < PF_BN / 16; ++k) {
-          const uint32_t a_off = (k / 4) * REGION + (k % 4) * 32;
-          tc::mma_ss(tmem + 2 * PF_BN, tc::desc_sw128(ps + a_off, 16, 1024),
+        for (int k = 0; k < PF_BN / 16; ++k)
+          tc::mma_ts(tmem + L::T_O + x * D, tmem + L::T_S + x * 128 + k * 8,
                      tc::desc_sw128(vs + k * 16 * 128, REGION, 1024), idesc_pv, !first_of_item || k > 0);
-        }
-        tc::commit(o_done);
-        tc::commit(&v_empty[st]);
         return true;
       };
       for (long long item = first; ok && item < a.num_items; item += stride) {
         const PrefillItem it = prefill_item(a, item);
         if (!it.work) continue;
-        const int qb = n_items & 1;
-        if (!(ok = mbar_wait_bounded(&q_full[qb], (uint32_t)((n_items >> 1) & 1), limit))) break;
-        const uint32_t qs = sbase + L::Q + qb * HALVES * REGION;
+        if (!(ok = mbar_wait_bounded(q_full, (uint32_t)(n_items & 1), limit))) break;
+        long long pend_t = -1, pend_tb = 0;  // PV_B due next: K/V tile and B's tile
+        bool pend_first = false;
         for (int j = 0; j < it.nt; ++j, ++g) {
           if (*abort_flag) {
             ok = false;
             break;
           }
-          const int st = (int)(g % PF_KST);
-          if (!(ok = mbar_wait_bounded(&k_full[st], (uint32_t)((g / PF_KST) & 1), limit))) break;
+          const bool a_on = j < it.nt_a, b_on = it.has_b;
+          if (!(ok = mbar_wait_bounded(&k_full[g % PF_KST], (uint32_t)((g / PF_KST) & 1), limit))) break;
           tc::fence_after_sync();
-          const uint32_t ks = sbase + L::K + st * HALVES * REGION;
-          const uint32_t d = tmem + (uint32_t)(g & 1) * PF_BN;
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k / 4) * REGION + (k % 4) * 32;
-            tc::mma_ss(d, tc::desc_sw128(qs + off, 16, 1024), tc::desc_sw128(ks + off, 16, 1024), idesc_qk, k > 0);
+          if (a_on) issue_qk(0, g);
+          if (pend_t >= 0) {
+            if (!(ok = issue_pv(1, pend_t, pend_tb, pend_first))) break;
+            tc::commit(&v_empty[pend_t % PF_VST]);
+            pend_t = -1;
           }
-          tc::commit(&s_full[g & 1]);
-          tc::commit(&k_empty[st]);
-          if (j == it.nt - 1) tc::commit(&q_empty[qb]);
-          if (pending >= 0 && !(ok = issue_pv(pending, pending_first))) break;
-          pending = g;
-          pending_first = j == 0;
+          if (b_on) issue_qk(1, g);
+          tc::commit(&k_empty[g % PF_KST]);
+          if (j == it.nt - 1) tc::commit(q_empty);
+          if (a_on) {
+            if (!(ok = issue_pv(0, g, gx[0], j == 0))) break;
+            if (j == it.nt_a - 1) tc::commit(&o_done[0]);
+            if (!b_on) tc::commit(&v_empty[g % PF_VST]);
+            ++gx[0];
+          }
+          if (b_on) {
+            pend_t = g;
+            pend_tb = gx[1]++;
+            pend_first = j == 0;
+          }
+        }
+        if (ok && pend_t >= 0) {  // the item's last PV_B
+          if ((ok = issue_pv(1, pend_t, pend_tb, pend_first))) {
+            tc::commit(&v_empty[pend_t % PF_VST]);
+            tc::commit(&o_done[1]);
+          }
         }
         ++n_items;
       }
-      if (ok && pending >= 0) ok = issue_pv(pending, pending_first);
       if (!ok) {
         *abort_flag = 1;
         atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
@@ -349,57 +378,58 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       if (!mbar_wait_bounded(drained, 0, limit)) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
     }
   } else {
-    // ------------------------------------------------------------ softmax and epilogue (warps 0-3, one row each)
-    const int r = warp * 32 + lane;
-    const uint32_t lanes = (uint32_t)(warp * 32) << 16;
-    long long g = 0;
-    int n_items = 0;
+    // ------------------------------------------------------------ softmax and epilogue of sub-tile x (warps 0-3: A, 4-7: B)
+    const int x = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lanes + L::T_S + x * 128, t_o = tmem + lanes + L::T_O + x * D;
+    long long g = 0;   // K/V tiles
+    long long gx = 0;  // this sub-tile's tiles
+    int n_items = 0, nx_items = 0;
     bool ok = true;
     for (long long item = first; ok && item < a.num_items; item += stride) {
       const PrefillItem it = prefill_item(a, item);
       if (it.bad_ctx) {
-        if (r == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
-        if (r < it.rows) {
-          uint4 *dst = reinterpret_cast<uint4 *>(a.out + (long long)(it.q0 + it.t0 + r) * a.out_token_stride +
+        if (r == 0 && x == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
+        if (x * PF_BM + r < it.rows) {
+          uint4 *dst = reinterpret_cast<uint4 *>(a.out + (long long)(it.q0 + it.t0 + x * PF_BM + r) * a.out_token_stride +
                                                  (long long)it.hq * D);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
         }
       }
       if (!it.work) continue;
+      const int ntx = x == 0 ? it.nt_a : (it.has_b ? it.nt : 0);
+      const bool zeroes_v = x == 0 ? it.nt_a == it.nt : it.nt_a < it.nt;  // first PV reader of the last tile
       // last key this row sees; rows past the item's tokens stop at kmax - 1 too, so that no row
       // reads a page the producers did not load
-      const int vis = min(it.pos0 + r, it.kmax - 1);
-      const int vis_min = min(it.pos0, it.kmax - 1);  // the smallest vis of the item's rows
+      const int pos0 = it.pos0 + x * PF_BM;
+      const int vis = min(pos0 + r, it.kmax - 1);
+      const int vis_min = min(pos0, it.kmax - 1);
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < it.nt; ++j, ++g) {
+      for (int j = 0; j < ntx; ++j, ++gx) {
         if (__any_sync(FULL, *abort_flag != 0)) {
           ok = false;
           break;
         }
-        if (!(ok = warp_wait(&s_full[g & 1], (uint32_t)((g >> 1) & 1), limit))) break;
+        // S_x(j) is in tensor memory, and every earlier MMA (PV_x of the previous tile) is done
+        if (!(ok = warp_wait(&s_full[x], (uint32_t)(gx & 1), limit))) break;
         tc::fence_after_sync();
-        float sv[PF_BN];
+        const int key0 = j * PF_BN;
+        const bool masked = key0 + PF_BN - 1 > vis_min;  // a tile on the diagonal or at the end (uniform)
+        // pass 1: row max of the raw scores (scale_log2 > 0 keeps the order)
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < PF_BN / 32; ++c) {
           float t[32];
-          tc::ld32(tmem + lanes + (uint32_t)(g & 1) * PF_BN + c * 32, t);
+          tc::ld32(t_s + c * 32, t);
+          tc::wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = t[i];
+          for (int i = 0; i < 32; ++i) {
+            const float v = (masked && key0 + c * 32 + i > vis) ? -INFINITY : t[i];
+            mx4[i & 3] = fmaxf(mx4[i & 3], v);
+          }
         }
-        tc::wait_ld();
-        const int key0 = j * PF_BN;
-        if (key0 + PF_BN - 1 > vis_min) {  // a tile on the diagonal or at the end: mask (uniform branch)
-#pragma unroll
-          for (int c = 0; c < PF_BN; ++c)
-            if (key0 + c > vis) sv[c] = -INFINITY;
-        }
-        // row max of the raw scores in four independent chains (scale_log2 > 0 keeps the order)
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < PF_BN; c += 4)
-#pragma unroll
-          for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], sv[c + u]);
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
         const float m_new = fmaxf(m, mx);
         const bool need = m_new > m + RESCALE_SLACK;
@@ -408,75 +438,84 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           factor = ex2(m - m_new);
           m = m_new;
         }
-        // p = 2^(s * scale_log2 - m): one FFMA and one SFU op per score; fp32 sums in four chains
-        uint32_t pk[PF_BN / 2];
+        // pass 2: p = 2^(s * scale_log2 - m), rounded to the storage type, into P_x (the first 64
+        // columns of S_x: chunk c's 16 packed columns overlap only scores already read)
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < PF_BN / 2; ++c) {
-          const float p0 = ex2(fmaf(sv[2 * c], a.scale_log2, -m));
-          const float p1 = ex2(fmaf(sv[2 * c + 1], a.scale_log2, -m));
-          sum4[(2 * c) & 3] += p0;
-          sum4[(2 * c + 1) & 3] += p1;
-          pk[c] = E::narrow2(p0, p1);
+        for (int c = 0; c < PF_BN / 32; ++c) {
+          float t[32];
+          tc::ld32(t_s + c * 32, t);
+          tc::wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k0 = key0 + c * 32 + 2 * i;
+            const float p0 = (masked && k0 > vis) ? 0.f : ex2(fmaf(t[2 * i], a.scale_log2, -m));
+            const float p1 = (masked && k0 + 1 > vis) ? 0.f : ex2(fmaf(t[2 * i + 1], a.scale_log2, -m));
+            sum4[(2 * i) & 3] += p0;
+            sum4[(2 * i + 1) & 3] += p1;
+            pk[i] = E::narrow2(p0, p1);
+          }
+          tc::st16(t_s + c * 16, pk);
         }
         const float rowsum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        if (j > 0 && __any_sync(FULL, need)) {  // O_x is settled: the previous PV_x is done
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tc::ld32(t_o + c * 32, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= factor;
+            tc::st32(t_o + c * 32, o);
+          }
+        }
+        tc::wait_st();
+        l = l * factor + rowsum;
         if (j == it.nt - 1) {
           // The V producer publishes the item's missing pages with this tile's arrival.  V rows from
           // kmax on are past the context (whatever the pool holds there, possibly NaN) or in pages
-          // never loaded (stale smem); P is 0 for them but 0 * NaN is not, so they are zeroed.
+          // never loaded (stale smem); P is 0 for them but 0 * NaN is not, so the sub-tile whose PV
+          // reads the last tile first zeroes them.
           const int st = (int)(g % PF_VST);
           if (!(ok = warp_wait(&v_full[st], (uint32_t)((g / PF_VST) & 1), limit))) break;
-          if (key0 + PF_BN > it.kmax && key0 + r >= it.kmax) {
+          if (zeroes_v && key0 + PF_BN > it.kmax && key0 + r >= it.kmax) {
 #pragma unroll
             for (int hh = 0; hh < HALVES; ++hh) {
               uint4 *row = reinterpret_cast<uint4 *>(sm + L::V + (st * HALVES + hh) * REGION + r * 128);
 #pragma unroll
               for (int c = 0; c < 8; ++c) row[c] = make_uint4(0, 0, 0, 0);
             }
+            fence_proxy_async_smem();
           }
         }
-        if (g > 0) {  // the previous PV has read P (and, within an item, O is settled)
-          if (!(ok = warp_wait(o_done, (uint32_t)((g - 1) & 1), limit))) break;
-          tc::fence_after_sync();
-          if (j > 0 && __any_sync(FULL, need)) {
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              float o[32];
-              tc::ld32(tmem + lanes + 2 * PF_BN + c * 32, o);
-              tc::wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] *= factor;
-              tc::st32(tmem + lanes + 2 * PF_BN + c * 32, o);
-            }
-            tc::wait_st();
-          }
-        }
-        l = l * factor + rowsum;
-        // P row r, 128-byte swizzle: 16-byte chunk c of a 128-byte row goes to chunk c ^ (r & 7).
-#pragma unroll
-        for (int c = 0; c < PF_BN / 8; ++c) {
-          uint4 *dst = reinterpret_cast<uint4 *>(sm + L::P + (c / 8) * REGION + r * 128 + (((c % 8) ^ (r & 7)) * 16));
-          *dst = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
         tc::fence_before_sync();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[x]);
+        ++g;
       }
       if (!ok) break;
-      // epilogue: O after the item's last PV, normalised
-      if (!(ok = warp_wait(o_done, (uint32_t)((g - 1) & 1), limit))) break;
+      g += it.nt - ntx;  // tiles this sub-tile does not read
+      if (ntx == 0) {
+        ++n_items;
+        continue;
+      }
+      if (ntx < it.nt) {  // sub-tile A skips the last tiles: it still needs the item's missing-page flag
+        const long long gl = g - 1;
+        if (!(ok = warp_wait(&v_full[gl % PF_VST], (uint32_t)((gl / PF_VST) & 1), limit))) break;
+      }
+      // epilogue: O_x after the item's last PV_x, normalised
+      if (!(ok = warp_wait(&o_done[x], (uint32_t)(nx_items & 1), limit))) break;
       tc::fence_after_sync();
       const bool zero = bad_pages[n_items & 3] != 0;
-      __syncwarp();
-      if (r == 0) bad_pages[n_items & 3] = 0;  // free the slot for item n_items + 4
-      uint16_t *dst = a.out + (long long)(it.q0 + it.t0 + r) * a.out_token_stride + (long long)it.hq * D;
+      const int row = x * PF_BM + r;
+      uint16_t *dst = a.out + (long long)(it.q0 + it.t0 + row) * a.out_token_stride + (long long)it.hq * D;
       const float inv = 1.f / l;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
-        tc::ld32(tmem + lanes + 2 * PF_BN + c * 32, o);  // every lane: the load is warp-collective
+        tc::ld32(t_o + c * 32, o);  // every lane: the load is warp-collective
         tc::wait_ld();
-        if (r < it.rows) {
+        if (row < it.rows) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float f[8];
@@ -488,6 +527,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       tc::fence_before_sync();
       ++n_items;
+      ++nx_items;
     }
     if (!ok) {
       *abort_flag = 1;
@@ -496,7 +536,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 10) {
     __syncwarp();
     tc::fence_after_sync();
     tc::dealloc(tmem, PF_TMEM_COLS);
