@@ -12,8 +12,8 @@
 //   S_x = Q_x K^T    tcgen05.mma M=128 N=128 K=d, Q and K from swizzled smem,
 //                    S_x in tensor memory;
 //   softmax_x        one warpgroup per sub-tile, one row per thread: S_x read
-//                    from tensor memory (twice: max, then exponentials),
-//                    causal mask, online max with a lazy rescale of O_x, P_x
+//                    from tensor memory into registers (four loads, one
+//                    wait), causal mask, online max with a lazy rescale of O_x, P_x
 //                    rounded to the storage type and stored back into the
 //                    first half of S_x's columns;
 //   O_x += P_x V     tcgen05.mma M=128 N=d K=128 with P_x read from tensor
@@ -417,19 +417,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         tc::fence_after_sync();
         const int key0 = j * PF_BN;
         const bool masked = key0 + PF_BN - 1 > vis_min;  // a tile on the diagonal or at the end (uniform)
-        // pass 1: row max of the raw scores (scale_log2 > 0 keeps the order)
+        // the row of S_x: four loads, one wait
+        float sv[PF_BN];
+#pragma unroll
+        for (int c = 0; c < PF_BN / 32; ++c) tc::ld32(t_s + c * 32, *reinterpret_cast<float(*)[32]>(&sv[c * 32]));
+        tc::wait_ld();
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < PF_BN; ++c)
+            if (key0 + c > vis) sv[c] = -INFINITY;
+        }
+        // row max of the raw scores in four chains (scale_log2 > 0 keeps the order)
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < PF_BN / 32; ++c) {
-          float t[32];
-          tc::ld32(t_s + c * 32, t);
-          tc::wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float v = (masked && key0 + c * 32 + i > vis) ? -INFINITY : t[i];
-            mx4[i & 3] = fmaxf(mx4[i & 3], v);
-          }
-        }
+        for (int c = 0; c < PF_BN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], sv[c]);
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
         const float m_new = fmaxf(m, mx);
         const bool need = m_new > m + RESCALE_SLACK;
@@ -438,20 +439,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           factor = ex2(m - m_new);
           m = m_new;
         }
-        // pass 2: p = 2^(s * scale_log2 - m), rounded to the storage type, into P_x (the first 64
-        // columns of S_x: chunk c's 16 packed columns overlap only scores already read)
+        // p = 2^(s * scale_log2 - m) (0 where masked), rounded to the storage type, into P_x: the
+        // first 64 columns of S_x, whose scores are all in registers by now
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < PF_BN / 32; ++c) {
-          float t[32];
-          tc::ld32(t_s + c * 32, t);
-          tc::wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int k0 = key0 + c * 32 + 2 * i;
-            const float p0 = (masked && k0 > vis) ? 0.f : ex2(fmaf(t[2 * i], a.scale_log2, -m));
-            const float p1 = (masked && k0 + 1 > vis) ? 0.f : ex2(fmaf(t[2 * i + 1], a.scale_log2, -m));
+            const float s0 = sv[c * 32 + 2 * i], s1 = sv[c * 32 + 2 * i + 1];
+            const float p0 = s0 == -INFINITY ? 0.f : ex2(fmaf(s0, a.scale_log2, -m));
+            const float p1 = s1 == -INFINITY ? 0.f : ex2(fmaf(s1, a.scale_log2, -m));
             sum4[(2 * i) & 3] += p0;
             sum4[(2 * i + 1) & 3] += p1;
             pk[i] = E::narrow2(p0, p1);
