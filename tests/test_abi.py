@@ -103,3 +103,55 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(pa.PagedAttentionError):
         pa.decode(x, x, x, torch.zeros(2, 1, dtype=torch.int32), torch.zeros(2, dtype=torch.int32), 0.1,
                   max_context_len=1)
+
+
+def _prefill(lib, **over):
+    args = dict(q=16, k=16, v=16, bt=16, qs=16, cl=16, scale=0.1, out=16, S=2, N=40, hq=4, hkv=2, d=128, bs=16,
+                nb=10, mb=4, mql=32, qts=512, ots=512, dtype=1, stream=None)
+    args.update(over)
+    return lib.pa_prefill(args["q"], args["k"], args["v"], args["bt"], args["qs"], args["cl"], args["scale"],
+                          args["out"], args["S"], args["N"], args["hq"], args["hkv"], args["d"], args["bs"],
+                          args["nb"], args["mb"], args["mql"], args["qts"], args["ots"], args["dtype"], args["stream"])
+
+
+def test_host_validation_of_prefill(lib):
+    assert _prefill(lib, d=96) == -5
+    assert _prefill(lib, bs=8) == -5
+    assert _prefill(lib, hq=6, hkv=4) == -6
+    assert _prefill(lib, dtype=0) == -2
+    assert _prefill(lib, S=-1) == -3
+    assert _prefill(lib, mql=-1) == -3
+    assert _prefill(lib, qts=100) == -3  # token stride shorter than a token's heads
+    assert _prefill(lib, scale=float("nan")) == -3
+    assert _prefill(lib, out=None) == -1
+    assert _prefill(lib, q=24) == -4
+    assert _prefill(lib, ots=516) == -4
+    assert _prefill(lib, nb=0) == -3  # an empty pool has no rows for the tensor maps
+    assert _prefill(lib, S=0) == 0 and _prefill(lib, N=0) == 0 and _prefill(lib, mql=0) == 0
+
+
+def test_host_validation_of_block_copies(lib):
+    c = lib.pa_copy_blocks
+    # (k, v, mapping, n, hkv, d, bs, nb, stream)
+    assert c(16, 16, 16, 3, 4, 96, 16, 10, None) == -5
+    assert c(16, 16, 16, 3, 4, 128, 8, 10, None) == -5
+    assert c(16, 16, 16, -1, 4, 128, 16, 10, None) == -3
+    assert c(16, 16, 16, 3, 0, 128, 16, 10, None) == -3
+    assert c(None, 16, 16, 3, 4, 128, 16, 10, None) == -1
+    assert c(16, 16, None, 3, 4, 128, 16, 10, None) == -1
+    assert c(24, 16, 16, 3, 4, 128, 16, 10, None) == -4
+    assert c(16, 16, 20, 3, 4, 128, 16, 10, None) == -4  # mapping must be 8-byte aligned
+    assert c(16, 16, 16, 0, 4, 128, 16, 10, None) == 0  # nothing to copy: no CUDA call
+    s = lib.pa_swap_blocks
+    # (src_k, src_v, dst_k, dst_v, mapping, n, hkv, d, bs, src_nb, dst_nb, stream)
+    assert s(16, 16, 16, 16, 16, 2, 4, 128, 16, 10, 0, None) == -3
+    assert s(16, 16, 16, 16, 16, 2, 4, 64, 32, 10, 10, None) != -5  # d 64 and bs 32 are supported
+    assert s(16, 16, 16, 16, 16, 0, 4, 64, 32, 10, 10, None) == 0
+    if not _has_gpu():
+        # valid arguments reach the pointer check, which needs the CUDA runtime: reported, not thrown
+        assert s(16, 16, 16, 16, 16, 2, 4, 64, 32, 10, 10, None) in (-9, -11)
+
+
+def test_status_strings_cover_new_codes(lib):
+    for code in (-10, -11):
+        assert lib.pa_status_string(code) != b"unknown status"
