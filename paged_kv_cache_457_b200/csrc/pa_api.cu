@@ -644,6 +644,33 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, i
                         block_size, num_blocks, num_blocks, stream);
 }
 
+// Work counters of pa_prefill calls: a call takes the next of 64 slots and zeroes it on its own stream
+// before the launch, so calls in flight on different streams (up to 64) never share a counter.
+static __device__ unsigned int g_prefill_queue[64];
+void *g_prefill_queue_addr[kMaxDevices] = {};
+std::atomic<uint32_t> g_prefill_slot{0};
+
+int prefill_queue_slot(unsigned int **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record(e);
+  if (dev < 0 || dev >= kMaxDevices) {
+    t_last_cuda_error = "device ordinal beyond the library's table";
+    return PA_ERR_CUDA;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_prefill_queue_addr[dev]) {
+      void *p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_prefill_queue);
+      if (e != cudaSuccess) return record(e);
+      g_prefill_queue_addr[dev] = p;
+    }
+  }
+  *out = static_cast<unsigned int *>(g_prefill_queue_addr[dev]) + g_prefill_slot.fetch_add(1) % 64;
+  return PA_OK;
+}
+
 int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
                const int32_t *query_start, const int32_t *context_lens, float scale, void *out, int32_t num_seqs,
                int64_t num_query_tokens, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
@@ -714,6 +741,11 @@ int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const in
   // persistent: one CTA per SM (the shared-memory footprint admits no second one)
   const dim3 grid((unsigned)std::min<long long>(a.num_items, sms));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a.num_items > 0xffffffffLL) return PA_ERR_SHAPE;
+  rc = prefill_queue_slot(&a.queue);
+  if (rc != PA_OK) return rc;
+  cudaError_t me = cudaMemsetAsync(a.queue, 0, sizeof(unsigned int), st);
+  if (me != cudaSuccess) return record(me);
   auto launch = [&](auto kernel, uint32_t smem) -> int {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return record(e);

@@ -4,10 +4,10 @@
 //
 // Work item: 256 consecutive new tokens of one sequence for one query head,
 // as two 128-row sub-tiles A and B that share every K/V tile (half the K/V
-// bytes per flop of one 128-row tile).  Persistent CTAs (one per SM) walk the
-// items round-robin; the items of one (sequence, head) are adjacent, so the
-// CTAs working on them at the same time share that head's K/V through L2, and
-// the latest (heaviest) query tiles come first.  Per key tile of 128 tokens
+// bytes per flop of one 128-row tile).  Persistent CTAs (one per SM) take
+// items from a per-call counter, latest (heaviest) query tiles of every
+// sequence first; the producer warp fetches each item and hands it to the
+// other roles through a 4-deep ring in shared memory.  Per key tile of 128 tokens
 // (8 pages of 16 or 4 of 32), for each sub-tile x:
 //   S_x = Q_x K^T    tcgen05.mma M=128 N=128 K=d, Q and K from swizzled smem,
 //                    S_x in tensor memory;
@@ -43,6 +43,7 @@ struct PrefillArgs {
   const int32_t *query_start;   // [num_seqs + 1]
   const int32_t *context_lens;  // [num_seqs], new tokens included
   uint16_t *out;                // [num_query_tokens][num_q_heads][head_dim]
+  unsigned int *queue;          // work counter of this call, zero at launch
   long long num_blocks, out_token_stride, num_query_tokens, num_items;
   unsigned long long wait_limit_ns;
   float scale_log2;
@@ -56,6 +57,7 @@ constexpr int PF_THREADS = 11 * 32;
 constexpr int PF_KST = 3;              // K ring
 constexpr int PF_VST = 2;              // V ring
 constexpr uint32_t PF_TMEM_COLS = 512;
+constexpr int PF_ITEM_READERS = 10;  // V producer, MMA lane, 8 softmax warps
 
 template <int D>
 struct PrefillSmem {
@@ -65,7 +67,8 @@ struct PrefillSmem {
   static constexpr uint32_t K = Q + 2 * HALVES * REGION;
   static constexpr uint32_t V = K + PF_KST * HALVES * REGION;
   static constexpr uint32_t BARS = V + PF_VST * HALVES * REGION;
-  static constexpr uint32_t BYTES = BARS + 256;
+  // 27 mbarriers, the item ring, the tensor-memory address and flags: 272 bytes used
+  static constexpr uint32_t BYTES = BARS + 512;
   // + alignment slack; at least 120 KB so that one CTA holds an SM (and its tensor memory) alone
   static constexpr uint32_t ALLOC = (BYTES + 1024 > 120 * 1024) ? BYTES + 1024 : 120 * 1024;
   // tensor memory columns
@@ -89,25 +92,26 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
 // One work item as every role sees it (all values uniform across the CTA).
 struct PrefillItem {
   int s, hq, h, q0, t0, rows, ctx, pos0, kmax, nt, nt_a;
-  bool work, bad_ctx, has_b;
+  bool work, bad_ctx, bad_rows, has_b;
 };
 
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillArgs &a, long long item) {
   PrefillItem it;
-  const int per_seq = a.q_tiles * a.num_q_heads;
-  it.s = (int)(item / per_seq);
-  const int rem = (int)(item - (long long)it.s * per_seq);
-  it.hq = rem / a.q_tiles;
-  const int qt = a.q_tiles - 1 - rem % a.q_tiles;  // latest (heaviest) query tiles first
+  // item order: query tile (latest, i.e. heaviest, first), then sequence, then head
+  const long long per_tile = (long long)a.num_seqs * a.num_q_heads;
+  const int qt = a.q_tiles - 1 - (int)(item / per_tile);
+  const int rem = (int)(item % per_tile);
+  it.s = rem / a.num_q_heads;
+  it.hq = rem % a.num_q_heads;
   it.h = it.hq / (a.num_q_heads / a.num_kv_heads);
   it.q0 = a.query_start[it.s];
   const int n = a.query_start[it.s + 1] - it.q0;
   it.ctx = a.context_lens[it.s];
   it.t0 = qt * PF_ROWS;
-  it.work = it.bad_ctx = it.has_b = false;
+  it.work = it.bad_ctx = it.bad_rows = it.has_b = false;
   it.rows = it.pos0 = it.kmax = it.nt = it.nt_a = 0;
   if (it.q0 < 0 || n < 0 || (long long)it.q0 + n > a.num_query_tokens) {  // rows outside q / out
-    if (qt == a.q_tiles - 1 && it.hq == 0 && threadIdx.x == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
+    it.bad_rows = true;
     return it;
   }
   if (it.t0 >= n) return it;
@@ -164,6 +168,8 @@ __device__ __forceinline__ void load_tile(const PrefillArgs &a, const PrefillIte
   }
 }
 
+static_assert(PrefillSmem<128>::ALLOC <= 232448, "prefill smem over the per-block opt-in limit");
+
 template <class E, int D>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -190,7 +196,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   uint64_t *p_full = s_full + 2;        // [2]: P_A, P_B written
   uint64_t *o_done = p_full + 2;        // [2]: an item's last PV of A, of B done
   uint64_t *drained = o_done + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drained + 1);
+  uint64_t *item_full = drained + 1;   // [4]: the ring of items handed out by the producer warp
+  uint64_t *item_empty = item_full + 4;
+  volatile long long *items = reinterpret_cast<volatile long long *>(item_empty + 4);  // [4]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(const_cast<long long *>(items + 4));
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   volatile int *bad_pages = abort_flag + 1;  // [4]: per item, a ring of 4
 
@@ -212,6 +221,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       mbar_init(&o_done[i], 1);
     }
     mbar_init(drained, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&item_full[i], 1);
+      mbar_init(&item_empty[i], PF_ITEM_READERS);
+    }
     *abort_flag = 0;
     for (int i = 0; i < 4; ++i) bad_pages[i] = 0;
     fence_mbar_init();
@@ -225,7 +238,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const unsigned long long limit = a.wait_limit_ns;
-  const long long first = blockIdx.x, stride = gridDim.x;
+  // The k-th item the producer warp handed out (-1: none left), for one warp or one lane.
+  auto take_item = [&](int k, bool whole_warp, long long *idx) -> bool {
+    const int slot = k & 3;
+    const bool ok = whole_warp ? warp_wait(&item_full[slot], (uint32_t)((k >> 2) & 1), limit)
+                               : mbar_wait_bounded(&item_full[slot], (uint32_t)((k >> 2) & 1), limit);
+    *idx = items[slot];
+    if (whole_warp) __syncwarp();
+    if (!whole_warp || lane == 0) mbar_arrive(&item_empty[slot]);
+    return ok;
+  };
 
   if (warp == 8 || warp == 9) {
     // ------------------------------------------------------------ TMA producers: Q and K (warp 8), V (warp 9)
@@ -241,9 +263,44 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     long long g = 0;  // tiles issued so far
     int n_items = 0;
     bool ok = true;
-    for (long long item = first; ok && item < a.num_items; item += stride) {
-      const PrefillItem it = prefill_item(a, item);
-      if (!it.work) continue;
+    for (int k = 0; ok; ++k) {
+      long long item;
+      PrefillItem it;
+      if (is_k) {
+        // fetch the next item with work; items whose rows or context are invalid are settled here
+        const int slot = k & 3;
+        if (k >= 4 && !(ok = warp_wait(&item_empty[slot], (uint32_t)(((k >> 2) - 1) & 1), limit))) break;
+        for (;;) {
+          unsigned int t = 0;
+          if (lane == 0) t = atomicAdd(a.queue, 1u);
+          item = (long long)__shfl_sync(FULL, t, 0);
+          if (item >= a.num_items) {
+            item = -1;
+            break;
+          }
+          it = prefill_item(a, item);
+          if (it.work) break;
+          if (it.bad_rows && lane == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
+          if (it.bad_ctx) {  // zero the item's rows
+            if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
+            for (int r = lane; r < it.rows; r += 32) {
+              uint4 *dst = reinterpret_cast<uint4 *>(a.out + (long long)(it.q0 + it.t0 + r) * a.out_token_stride +
+                                                     (long long)it.hq * D);
+#pragma unroll
+              for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+        if (lane == 0) {
+          items[slot] = item;
+          mbar_arrive(&item_full[slot]);  // release: the item index is visible to the readers
+        }
+        if (item < 0) break;
+      } else {
+        if (!(ok = take_item(k, true, &item))) break;
+        if (item < 0) break;
+        it = prefill_item(a, item);
+      }
       if (is_k) {
         if (n_items >= 1 && !(ok = warp_wait(q_empty, (uint32_t)((n_items - 1) & 1), limit))) break;
         if (lane == 0) {
@@ -326,9 +383,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                      tc::desc_sw128(vs + k * 16 * 128, REGION, 1024), idesc_pv, !first_of_item || k > 0);
         return true;
       };
-      for (long long item = first; ok && item < a.num_items; item += stride) {
+      for (int k = 0; ok; ++k) {
+        long long item;
+        if (!(ok = take_item(k, false, &item))) break;
+        if (item < 0) break;
         const PrefillItem it = prefill_item(a, item);
-        if (!it.work) continue;
         if (!(ok = mbar_wait_bounded(q_full, (uint32_t)(n_items & 1), limit))) break;
         long long pend_t = -1, pend_tb = 0;  // PV_B due next: K/V tile and B's tile
         bool pend_first = false;
@@ -387,18 +446,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     long long gx = 0;  // this sub-tile's tiles
     int n_items = 0, nx_items = 0;
     bool ok = true;
-    for (long long item = first; ok && item < a.num_items; item += stride) {
+    for (int k = 0; ok; ++k) {
+      long long item;
+      if (!(ok = take_item(k, true, &item))) break;
+      if (item < 0) break;
       const PrefillItem it = prefill_item(a, item);
-      if (it.bad_ctx) {
-        if (r == 0 && x == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
-        if (x * PF_BM + r < it.rows) {
-          uint4 *dst = reinterpret_cast<uint4 *>(a.out + (long long)(it.q0 + it.t0 + x * PF_BM + r) * a.out_token_stride +
-                                                 (long long)it.hq * D);
-#pragma unroll
-          for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-        }
-      }
-      if (!it.work) continue;
       const int ntx = x == 0 ? it.nt_a : (it.has_b ? it.nt : 0);
       const bool zeroes_v = x == 0 ? it.nt_a == it.nt : it.nt_a < it.nt;  // first PV reader of the last tile
       // last key this row sees; rows past the item's tokens stop at kmax - 1 too, so that no row
