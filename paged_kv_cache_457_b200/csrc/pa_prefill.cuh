@@ -147,24 +147,21 @@ __device__ __forceinline__ int tile_page(const PrefillArgs &a, const PrefillItem
   return blk;
 }
 
-// Issues the TMA boxes of one key tile (K or V) into `dst`, completing on `bar`.
+// Issues the TMA boxes of one key tile (K or V) into `dst`, completing on `bar`: lane 0 posts the
+// expected bytes, then lane p issues the boxes of the tile's page p (its `blk`), so the pages' copies
+// go out together rather than one after another from a single thread.
 template <int HALVES>
 __device__ __forceinline__ void load_tile(const PrefillArgs &a, const PrefillItem &it, int blk, int lane,
                                           uint8_t *dst, const CUtensorMap *map, uint64_t *bar) {
   const int bs = a.block_size;
   const unsigned loaded = __ballot_sync(FULL, blk >= 0);
-  int ids[PF_BN / 16];
-#pragma unroll
-  for (int p = 0; p < PF_BN / 16; ++p) ids[p] = __shfl_sync(FULL, blk, p);
-  if (lane == 0) {
-    mbar_arrive_expect_tx(bar, (uint32_t)__popc(loaded) * bs * 128u * HALVES);
-    for (int p = 0; p < PF_BN / bs; ++p) {
-      if (!((loaded >> p) & 1u)) continue;
-      const long long row = ((long long)ids[p] * a.num_kv_heads + it.h) * bs;
-      for (int hh = 0; hh < HALVES; ++hh)
-        for (int b = 0; b < bs / TILE; ++b)
-          tma_load_2d(dst + hh * 128 * 128 + (p * bs + b * TILE) * 128, map, hh * 64, (int)(row + b * TILE), bar);
-    }
+  if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)__popc(loaded) * bs * 128u * HALVES);
+  __syncwarp();
+  if (blk >= 0) {
+    const long long row = ((long long)blk * a.num_kv_heads + it.h) * bs;
+    for (int hh = 0; hh < HALVES; ++hh)
+      for (int b = 0; b < bs / TILE; ++b)
+        tma_load_2d(dst + hh * 128 * 128 + (lane * bs + b * TILE) * 128, map, hh * 64, (int)(row + b * TILE), bar);
   }
 }
 
@@ -303,14 +300,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       if (is_k) {
         if (n_items >= 1 && !(ok = warp_wait(q_empty, (uint32_t)((n_items - 1) & 1), limit))) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full, 2 * PF_BM * D * 2);
-#pragma unroll
-          for (int x = 0; x < 2; ++x)
-#pragma unroll
-            for (int hh = 0; hh < HALVES; ++hh)
-              tc::tma_load_3d(sm + L::Q + (x * HALVES + hh) * REGION, &tmap_q, hh * 64, it.hq,
-                              it.q0 + it.t0 + x * PF_BM, q_full);
+        if (lane == 0) mbar_arrive_expect_tx(q_full, 2 * PF_BM * D * 2);
+        __syncwarp();
+        if (lane < 2 * HALVES) {  // lane = sub-tile * HALVES + half
+          const int x = lane / HALVES, hh = lane % HALVES;
+          tc::tma_load_3d(sm + L::Q + lane * REGION, &tmap_q, hh * 64, it.hq, it.q0 + it.t0 + x * PF_BM, q_full);
         }
       }
       bool any_bad = false;
@@ -492,16 +486,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           m = m_new;
         }
         // p = 2^(s * scale_log2 - m) (0 where masked), rounded to the storage type, into P_x: the
-        // first 64 columns of S_x, whose scores are all in registers by now
+        // first 64 columns of S_x, whose scores are all in registers by now.
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < PF_BN / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float s0 = sv[c * 32 + 2 * i], s1 = sv[c * 32 + 2 * i + 1];
-            const float p0 = s0 == -INFINITY ? 0.f : ex2(fmaf(s0, a.scale_log2, -m));
-            const float p1 = s1 == -INFINITY ? 0.f : ex2(fmaf(s1, a.scale_log2, -m));
+            // masked scores are -inf: 2^-inf = 0
+            const float p0 = ex2(fmaf(sv[c * 32 + 2 * i], a.scale_log2, -m));
+            const float p1 = ex2(fmaf(sv[c * 32 + 2 * i + 1], a.scale_log2, -m));
             sum4[(2 * i) & 3] += p0;
             sum4[(2 * i + 1) & 3] += p1;
             pk[i] = E::narrow2(p0, p1);
