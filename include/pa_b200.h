@@ -174,9 +174,12 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
  *   context_lens int32 [num_seqs];
  *   out          like q, token stride out_token_stride;
  *   max_query_len >= every n_s (sizes the grid; rows past it are not computed).
- * Runs on the tensor cores (tcgen05, tensor memory accumulators), 128 new
- * tokens of one query head per CTA; computes in fp32 with P rounded to the
- * storage type.  Device-side errors: L_s < n_s or L_s > block_table_stride *
+ * Runs on the tensor cores (tcgen05, tensor memory accumulators): work items
+ * of 256 new tokens of one query head, taken from a per-call queue by
+ * persistent CTAs; computes in fp32 with P rounded to the storage type.
+ * Sequences with one new token cost a whole 128-row tile each here: batch
+ * them through pa_decode; sequences with none cost a few microseconds per
+ * thousand (query tile, head) slots of max_query_len.  Device-side errors: L_s < n_s or L_s > block_table_stride *
  * block_size -> PA_DEV_ERR_CONTEXT and zero rows; query_start entries that
  * leave [0, num_query_tokens] -> PA_DEV_ERR_CONTEXT and that sequence is not
  * written; a needed table entry outside the pool -> PA_DEV_ERR_BLOCK_ID and

@@ -277,7 +277,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           }
           it = prefill_item(a, item);
           if (it.work) break;
-          if (it.bad_rows && lane == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
+          if (!it.bad_ctx && lane == 0) {
+            // no rows of this sequence at this query tile (or no valid rows at all): the same holds for
+            // the sequence's remaining heads, which are the next items; move the counter past them
+            atomicMax(a.queue, (unsigned int)(item + a.num_q_heads - it.hq));
+            if (it.bad_rows) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
+          }
           if (it.bad_ctx) {  // zero the item's rows
             if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
             for (int r = lane; r < it.rows; r += 32) {

@@ -128,3 +128,43 @@ def test_full_size_sampled(name):
                                "query_start": np.array([0, qs[s + 1] - qs[s]], np.int32),
                                "context_lens": lens[s:s + 1], "block_tables": case.block_tables[s:s + 1]})
         compare(got[qs[s]:qs[s + 1]], expect(sub), case.dtype, what=f"{name} sequence {s}")
+
+
+def test_skewed_batch_one_long_prompt_among_decode_steps():
+    """A chunked-prefill batch: one long prompt and many one-token sequences (exact), and one prompt among
+    thousands of sequences with no new token, whose empty (query tile, sequence, head) items cost little."""
+    require_gpu()
+    shape = [(int(L), 1) for L in np.random.default_rng(15).integers(1, 300, size=120)] + [(2000, 2000)]
+    case = W.prefill_case(15, shape, 8, 2, 128, 16, "bf16")
+    got = run(case)
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+    compare(got[:120], expect(W.PrefillCase(**{**case.__dict__, "q": case.q[:120],
+                                                 "query_start": case.query_start[:121],
+                                                 "context_lens": case.context_lens[:120],
+                                                 "block_tables": case.block_tables[:120]})), "bf16",
+            what="one-token sequences")
+    last = W.PrefillCase(**{**case.__dict__, "q": case.q[120:], "query_start": np.array([0, 2000], np.int32),
+                            "context_lens": case.context_lens[120:], "block_tables": case.block_tables[120:]})
+    compare(got[120:], expect(last), "bf16", what="long prompt")
+    # empty items are cheap but not free: 4000 cached sequences that bring no new token and one 1000-token
+    # prompt, 8 query heads: 4 * 4001 * 8 items, all but 32 of them empty (about 0.7 ms on a B200; the bound
+    # catches a schedule that would spend a full item's pipeline on each)
+    big_shape = [(int(L), 0) for L in np.random.default_rng(16).integers(1, 64, size=4000)] + [(1000, 1000)]
+    big = W.prefill_case(16, big_shape, 8, 2, 128, 16, "bf16")
+    kc, vc = to_dev(big.k_cache, "bf16"), to_dev(big.v_cache, "bf16")
+    args = (to_dev(big.q, "bf16"), kc, vc, to_dev_index(big.block_tables), to_dev_index(big.query_start),
+            to_dev_index(big.context_lens), big.scale, big.max_query_len)
+    out = pa.prefill(*args)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(5):
+        pa.prefill(*args)
+    e1.record()
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+    assert e0.elapsed_time(e1) / 5 < 2.0
+    got_big = host_bits(out)
+    sub = W.PrefillCase(**{**big.__dict__, "query_start": np.array([0, 1000], np.int32),
+                           "context_lens": big.context_lens[-1:], "block_tables": big.block_tables[-1:]})
+    compare(got_big, expect(sub), "bf16", what="the prompt among empty sequences")
