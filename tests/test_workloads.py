@@ -110,3 +110,42 @@ def test_unique_and_logical_bytes():
     assert unique < logical
     # the eight 64-block prefixes are counted once in the unique figure
     assert logical - unique >= 7 * 8 * 1024 * 8 * 128 * 2 * 2
+
+
+def test_prefill_case_structure():
+    shape = [(1, 1), (40, 8), (300, 129), (16, 0), (64, 64)]
+    c = W.prefill_case(3, shape, 8, 2, 64, 16, "bf16")
+    assert c.query_start.tolist() == [0, 1, 9, 138, 138, 202]
+    assert c.context_lens.tolist() == [1, 40, 300, 16, 64]
+    assert c.q.shape == (202, 8, 64) and c.q.dtype == np.uint16
+    assert c.max_query_len == 129
+    # attended (query, key) pairs: n (L - n) + n (n + 1) / 2 per sequence
+    assert c.attended_pairs == sum(n * (L - n) + n * (n + 1) // 2 for L, n in shape)
+    # every table entry a sequence needs is a distinct block of the pool; the rest is padding
+    used = []
+    for s, (L, _) in enumerate(shape):
+        nblk = -(-L // 16)
+        row = c.block_tables[s]
+        assert (row[:nblk] >= 0).all() and (row[:nblk] < c.num_blocks).all()
+        assert (row[nblk:] == W.TABLE_PAD).all()
+        used += row[:nblk].tolist()
+    assert len(used) == len(set(used))
+    # slots no sequence owns hold NaN; owned slots hold finite draws
+    owned = np.zeros((c.num_blocks, 16), dtype=bool)
+    for s, (L, _) in enumerate(shape):
+        for j in range(L):
+            owned[c.block_tables[s, j // 16], j % 16] = True
+    kc = c.k_cache.transpose(0, 2, 1, 3)  # [NB, bs, Hkv, d]
+    assert (kc[~owned] == W.NAN_BITS["bf16"]).all()
+    vals = (kc[owned].astype(np.uint32) << 16).view(np.float32)
+    assert np.isfinite(vals).all()
+
+
+def test_named_prefill_workloads_are_deterministic():
+    for name, make in W.PREFILL_NAMED.items():
+        a, b = make(), make()
+        assert a.name == name
+        assert np.array_equal(a.q, b.q) and np.array_equal(a.block_tables, b.block_tables)
+        assert np.array_equal(a.query_start, b.query_start) and np.array_equal(a.context_lens, b.context_lens)
+        assert (a.context_lens >= np.diff(a.query_start)).all()
+        assert a.max_query_len <= 2048
