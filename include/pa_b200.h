@@ -173,7 +173,9 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
  *                query_start[num_seqs] <= num_query_tokens;
  *   context_lens int32 [num_seqs];
  *   out          like q, token stride out_token_stride;
- *   max_query_len >= every n_s (sizes the grid; rows past it are not computed).
+ *   max_query_len >= every n_s (sizes the grid); a sequence with more new
+ *                tokens sets PA_DEV_ERR_CONTEXT_HINT and its rows past
+ *                max_query_len (rounded up to 256) are not written.
  * Runs on the tensor cores (tcgen05, tensor memory accumulators): work items
  * of 256 new tokens of one query head, taken from a per-call queue by
  * persistent CTAs; computes in fp32 with P rounded to the storage type.

@@ -92,7 +92,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
 // One work item as every role sees it (all values uniform across the CTA).
 struct PrefillItem {
   int s, hq, h, q0, t0, rows, ctx, pos0, kmax, nt, nt_a;
-  bool work, bad_ctx, bad_rows, has_b;
+  bool work, bad_ctx, bad_rows, has_b, past_grid;
 };
 
 __device__ __forceinline__ PrefillItem prefill_item(const PrefillArgs &a, long long item) {
@@ -108,12 +108,13 @@ __device__ __forceinline__ PrefillItem prefill_item(const PrefillArgs &a, long l
   const int n = a.query_start[it.s + 1] - it.q0;
   it.ctx = a.context_lens[it.s];
   it.t0 = qt * PF_ROWS;
-  it.work = it.bad_ctx = it.bad_rows = it.has_b = false;
+  it.work = it.bad_ctx = it.bad_rows = it.has_b = it.past_grid = false;
   it.rows = it.pos0 = it.kmax = it.nt = it.nt_a = 0;
   if (it.q0 < 0 || n < 0 || (long long)it.q0 + n > a.num_query_tokens) {  // rows outside q / out
     it.bad_rows = true;
     return it;
   }
+  it.past_grid = (long long)n > (long long)a.q_tiles * PF_ROWS;  // more new tokens than max_query_len covers
   if (it.t0 >= n) return it;
   it.rows = min(PF_ROWS, n - it.t0);
   if (it.ctx < n || (long long)it.ctx > (long long)a.table_stride * a.block_size) {
@@ -276,6 +277,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             break;
           }
           it = prefill_item(a, item);
+          if (it.past_grid && it.t0 == 0 && it.hq == 0 && lane == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT_HINT);
           if (it.work) break;
           if (!it.bad_ctx && lane == 0) {
             // no rows of this sequence at this query tile (or no valid rows at all): the same holds for

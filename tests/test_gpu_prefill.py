@@ -96,6 +96,18 @@ def test_bad_page_and_bad_context_zero_their_rows():
     compare(got[qs[2]:], expect(ok), "fp16", what="untouched sequence")
 
 
+def test_max_query_len_too_small_is_flagged():
+    require_gpu()
+    case = W.prefill_case(17, [(600, 600), (40, 40)], 4, 4, 64, 16, "fp16")
+    pa.device_status(clear=True)
+    got = run(case, max_query_len=200)  # covers 256 rows: sequence 0's rows 256.. are left unwritten
+    torch.cuda.synchronize()
+    assert pa.device_status() & pa.DEV_ERR_CONTEXT_HINT
+    ref = expect(case)
+    compare(got[:256], ref[:256], "fp16", what="rows the grid covers")
+    compare(got[600:], ref[600:], "fp16", what="the other sequence")
+
+
 def test_chunked_equals_whole_prompt():
     """A prompt processed as two chunks (the second over the cached first) gives the one-pass rows."""
     require_gpu()
