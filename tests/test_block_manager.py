@@ -327,3 +327,51 @@ def test_manager_plans_through_the_oracle_decode():
             want = oracle.decode(q[i:i + 1], ck, cv, np.arange(nblk, dtype=np.int32)[None], np.array([L], np.int32),
                                  0.125, dtype)
             assert np.array_equal(got[i:i + 1], want), f"sequence {sid}"
+
+
+def test_concurrent_calls_keep_the_pool_consistent():
+    """Calls on one manager from several host threads are serialised: after a storm of adds, forks,
+    appends and frees the reference counts still equal the tables that name each page."""
+    import threading
+    bm = pa.BlockManager(16, 4096)
+    errors = []
+
+    def worker(base):
+        rng = np.random.default_rng(base)
+        mine = []
+        try:
+            for i in range(300):
+                sid = base * 100000 + i
+                r = rng.random()
+                if r < 0.4 or not mine:
+                    bm.add_sequence(sid, int(rng.integers(0, 80)))
+                    mine.append(sid)
+                elif r < 0.6:
+                    bm.fork(int(rng.choice(mine)), sid)
+                    mine.append(sid)
+                elif r < 0.85:
+                    bm.append_slot(int(rng.choice(mine)))
+                else:
+                    victim = int(rng.choice(mine))
+                    bm.free_sequence(victim)
+                    mine.remove(victim)
+        except BlockManagerError as e:
+            if e.code != -21:  # running out of pages is allowed under contention; anything else is not
+                errors.append(e)
+        return mine
+
+    results = {}
+    threads = [threading.Thread(target=lambda b=b: results.__setitem__(b, worker(b))) for b in range(1, 7)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors
+    refs = np.zeros(4096, dtype=np.int64)
+    for mine in results.values():
+        for sid in mine:
+            t = bm.block_table(sid)
+            assert len(t) == -(-bm.num_tokens(sid) // 16)
+            np.add.at(refs, t, 1)
+    assert [bm.ref_count(b) for b in range(4096)] == refs.tolist()
+    assert bm.num_free_device_blocks == int((refs == 0).sum())
