@@ -370,9 +370,18 @@ int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  const long long warps = (long long)args.num_seqs * args.num_q_heads;
-  const int grid = (int)std::max(1LL, std::min<long long>((warps + 7) / 8, (long long)sms * 8));
-  e = launch_pdl(pa::decode_merge_kernel<E, D>, dim3(grid), dim3(256), 0, stream, args);
+  if (uses_mma(args.group)) {  // one warp per (sequence, query head), eight per block
+    const long long warps = (long long)args.num_seqs * args.num_q_heads;
+    const int grid = (int)std::max(1LL, std::min<long long>((warps + 7) / 8, (long long)sms * 8));
+    e = launch_pdl(pa::decode_merge_heads_kernel<E, D>, dim3(grid), dim3(256), 0, stream, args);
+  } else {  // one warp per segment (sequence, kv head: 1 or 2 query heads), two per block
+    const long long warps = (long long)args.num_seqs * args.num_kv_heads;
+    const dim3 mgrid((unsigned)((warps + 1) / 2)), mblock(64);
+    if (args.heads_per_unit == 2)
+      e = launch_pdl(pa::decode_merge_kernel<E, D, 2, 8>, mgrid, mblock, 0, stream, args);
+    else
+      e = launch_pdl(pa::decode_merge_kernel<E, D, 1, 16>, mgrid, mblock, 0, stream, args);
+  }
   if (e != cudaSuccess) return record(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);

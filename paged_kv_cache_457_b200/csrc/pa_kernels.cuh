@@ -699,14 +699,171 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
   }
 }
 
-// One warp per (sequence, query head): writes the zero rows of empty or
-// invalid sequences (setting the status bits of the invalid ones) and merges
-// the partial pieces of segments that the split kernel cut across chunks:
-// out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p, M = max_p m_p, summed
-// in increasing chunk order (deterministic).  Built for latency: lane p holds
-// piece p's (m, l) and weight, and the partial rows are loaded eight at a time.
+// One warp per HW query heads of a segment (sequence s, head chunk: G query heads of one kv head): writes
+// the zero rows of empty or invalid sequences (setting the status bits of the invalid ones) and merges the
+// partial pieces of segments that the split kernel cut across chunks:
+//   out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p,
+// summed in increasing chunk order (deterministic).  Built for latency, since it runs after the split grid
+// has drained: the pieces' (m, l) and the partial rows of the first MB pieces are requested together, so a
+// segment cut into at most MB pieces costs two dependent trips to memory after the wait (tile prefix, then
+// pieces).  Blocks of two warps, so registers, not block slots, bound the warps per SM.
+template <class E, int D, int HW, int MB>
+__global__ void __launch_bounds__(64) decode_merge_kernel(const DecodeArgs a) {
+  static_assert(32 % MB == 0, "a batch of pieces never straddles a 32-piece window");
+  constexpr int DPL = D / 32;  // dims per lane (4 or 2)
+  const int lane = threadIdx.x & 31;
+  grid_dependency_wait();  // the split kernel's pieces and tile prefix
+  grid_launch_dependents();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ws_queue = 0ull;  // leave the chunk counter clear
+  const int S = a.num_seqs;
+  const int HC = a.num_kv_heads * a.n_chunks;
+  const int G = a.heads_per_unit;
+  const int subs = G / HW;  // warps per segment
+  const long long w = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (w >= (long long)S * HC * subs) return;
+  const long long seg = w / subs;
+  const int gg0 = (int)(w - seg * subs) * HW;  // first head of this warp within the chunk
+  const int s = (int)(seg / HC);
+  const int hc = (int)(seg - (long long)s * HC);
+  const int L = __ldg(a.context_lens + s);
+  const int pt0 = __ldg(a.ws_tiles + s), pt1 = __ldg(a.ws_tiles + s + 1), pts = __ldg(a.ws_tiles + S);
+  uint16_t *dst =
+      a.out + (long long)s * a.out_seq_stride + (long long)(chunk_first_head(a, hc) + gg0) * D + lane * DPL;
+  float o[HW][DPL];
+#pragma unroll
+  for (int gg = 0; gg < HW; ++gg)
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) o[gg][k] = 0.f;
+  if (!context_ok(a, L) || L == 0) {
+    if (lane == 0 && L != 0 && hc == 0 && gg0 == 0)
+      atomicOr(&g_status, (L < 0 || (long long)L > (long long)a.table_stride * a.block_size) ? PA_DEV_ERR_CONTEXT
+                                                                                            : PA_DEV_ERR_CONTEXT_HINT);
+  } else {
+    const ChunkPlan plan = plan_chunks(a, pts);
+    const int nt = pt1 - pt0;
+    const long long seg0 = (long long)pt0 * HC + (long long)hc * nt;
+    const long long c_first = plan.chunk_of(seg0), c_last = plan.chunk_of(seg0 + nt - 1);
+    if (c_first == c_last) return;  // one chunk held the whole segment: the split kernel wrote the rows
+    const int n = (int)(c_last - c_first + 1);
+    auto piece_row = [&](int p) -> long long {  // partial row of this warp's first head in piece p
+      const long long c = c_first + p;
+      const int slot = (p == 0 && seg0 > plan.start(c)) ? 1 : 0;
+      return (c * 2 + slot) * G + gg0;
+    };
+    // (m, l) of the first 32 pieces (lane p holds piece p) and the partial rows of the first batch, together
+    float2 ml0[HW];
+#pragma unroll
+    for (int gg = 0; gg < HW; ++gg) ml0[gg] = make_float2(-INFINITY, 0.f);
+    if (lane < n) {
+      const long long r = piece_row(lane);
+#pragma unroll
+      for (int gg = 0; gg < HW; ++gg) ml0[gg] = __ldg(a.ws_ml + r + gg);
+    }
+    float t[MB][HW][DPL];
+    auto load_batch = [&](int base) {
+#pragma unroll
+      for (int i = 0; i < MB; ++i) {
+        const bool ok = base + i < n;
+        const long long r = ok ? piece_row(base + i) : 0;
+#pragma unroll
+        for (int gg = 0; gg < HW; ++gg) {
+          const float *src = a.ws_acc + (r + gg) * D + lane * DPL;
+          if constexpr (DPL == 4) {
+            const float4 v = ok ? __ldg(reinterpret_cast<const float4 *>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            t[i][gg][0] = v.x;
+            t[i][gg][1] = v.y;
+            t[i][gg][2] = v.z;
+            t[i][gg][3] = v.w;
+          } else {
+            const float2 v = ok ? __ldg(reinterpret_cast<const float2 *>(src)) : make_float2(0.f, 0.f);
+            t[i][gg][0] = v.x;
+            t[i][gg][1] = v.y;
+          }
+        }
+      }
+    };
+    load_batch(0);
+    // maximum and validity over all pieces, per head
+    float M[HW];
+    bool err = false;
+#pragma unroll
+    for (int gg = 0; gg < HW; ++gg) {
+      M[gg] = ml0[gg].x;
+      err |= lane < n && ml0[gg].y < 0.f;
+    }
+    for (int p = lane + 32; p < n; p += 32) {
+      const long long r = piece_row(p);
+#pragma unroll
+      for (int gg = 0; gg < HW; ++gg) {
+        const float2 ml = __ldg(a.ws_ml + r + gg);
+        M[gg] = fmaxf(M[gg], ml.x);
+        err |= ml.y < 0.f;
+      }
+    }
+#pragma unroll
+    for (int gg = 0; gg < HW; ++gg)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) M[gg] = fmaxf(M[gg], __shfl_xor_sync(FULL, M[gg], off));
+    if (!__any_sync(FULL, err)) {
+      // lane p of the current 32-piece window holds piece p's weight per head; the sum of weighted l runs per lane
+      float wt[HW], l[HW];
+#pragma unroll
+      for (int gg = 0; gg < HW; ++gg) {
+        wt[gg] = lane < n ? exp2f(ml0[gg].x - M[gg]) : 0.f;
+        l[gg] = ml0[gg].y * wt[gg];
+      }
+      for (int base = 0; base < n; base += MB) {
+        if (base > 0) {
+          if ((base & 31) == 0) {  // next window of 32 pieces: their (m, l)
+            const int p = base + lane;
+            const long long r = p < n ? piece_row(p) : 0;
+#pragma unroll
+            for (int gg = 0; gg < HW; ++gg) {
+              const float2 ml = p < n ? __ldg(a.ws_ml + r + gg) : make_float2(-INFINITY, 0.f);
+              wt[gg] = p < n ? exp2f(ml.x - M[gg]) : 0.f;
+              l[gg] = fmaf(ml.y, wt[gg], l[gg]);
+            }
+          }
+          load_batch(base);
+        }
+#pragma unroll
+        for (int i = 0; i < MB; ++i) {
+          const int src_lane = (base + i) & 31;
+#pragma unroll
+          for (int gg = 0; gg < HW; ++gg) {
+            const float wq = __shfl_sync(FULL, wt[gg], src_lane);  // 0 past the last piece
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) o[gg][k] = fmaf(wq, t[i][gg][k], o[gg][k]);
+          }
+        }
+      }
+#pragma unroll
+      for (int gg = 0; gg < HW; ++gg) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) l[gg] += __shfl_xor_sync(FULL, l[gg], off);
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) o[gg][k] = o[gg][k] / l[gg];
+      }
+    }
+  }
+#pragma unroll
+  for (int gg = 0; gg < HW; ++gg) {
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<uint2 *>(dst + gg * D) =
+          make_uint2(E::narrow2(o[gg][0], o[gg][1]), E::narrow2(o[gg][2], o[gg][3]));
+    } else {
+      *reinterpret_cast<uint32_t *>(dst + gg * D) = E::narrow2(o[gg][0], o[gg][1]);
+    }
+  }
+}
+
+// Merge for the tensor-core path: one warp per (sequence, query head), eight
+// warps per block, the same arithmetic and order as decode_merge_kernel (lane
+// p holds piece p's (m, l) and weight; partial rows are loaded eight at a
+// time once the maximum is known).  Measured faster than decode_merge_kernel
+// when a segment carries 3 to 8 heads.
 template <class E, int D>
-__global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(256) decode_merge_heads_kernel(const DecodeArgs a) {
   constexpr int DPL = D / 32;  // dims per lane (4 or 2)
   const int lane = threadIdx.x & 31;
   grid_dependency_wait();  // the split kernel's pieces and tile prefix

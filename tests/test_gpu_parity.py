@@ -76,6 +76,12 @@ SMALL = [  # (hq, hkv, d, bs, dtype)
     (12, 4, 64, 16, "fp16"),
     (16, 2, 128, 16, "bf16"),
     (2, 2, 128, 32, "bf16"),
+    (4, 2, 64, 16, "bf16"),     # group 2
+    (10, 2, 128, 16, "fp16"),   # group 5
+    (12, 2, 64, 32, "bf16"),    # group 6
+    (14, 2, 128, 16, "bf16"),   # group 7
+    (24, 2, 128, 16, "fp16"),   # group 12: two chunks of 6 heads per kv head
+    (32, 2, 64, 16, "bf16"),    # group 16: two chunks of 8 heads per kv head
 ]
 LENS = [1, 2, 15, 16, 17, 31, 33, 100, 257, 512, 513, 777, 1024, 1025]
 
