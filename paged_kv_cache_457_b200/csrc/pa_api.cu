@@ -345,7 +345,7 @@ int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, 
 }
 
 template <class E, int D>
-int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype, int sms, cudaStream_t stream) {
+int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype, cudaStream_t stream) {
   const int threads = kWarps * 32;
   if (uses_mma(args.group)) {
     const long long rows = args.num_blocks * args.num_kv_heads * args.block_size;
@@ -370,18 +370,17 @@ int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (uses_mma(args.group)) {  // one warp per (sequence, query head), eight per block
-    const long long warps = (long long)args.num_seqs * args.num_q_heads;
-    const int grid = (int)std::max(1LL, std::min<long long>((warps + 7) / 8, (long long)sms * 8));
-    e = launch_pdl(pa::decode_merge_heads_kernel<E, D>, dim3(grid), dim3(256), 0, stream, args);
-  } else {  // one warp per segment (sequence, kv head: 1 or 2 query heads), two per block
-    const long long warps = (long long)args.num_seqs * args.num_kv_heads;
-    const dim3 mgrid((unsigned)((warps + 1) / 2)), mblock(64);
-    if (args.heads_per_unit == 2)
-      e = launch_pdl(pa::decode_merge_kernel<E, D, 2, 8>, mgrid, mblock, 0, stream, args);
-    else
-      e = launch_pdl(pa::decode_merge_kernel<E, D, 1, 16>, mgrid, mblock, 0, stream, args);
-  }
+  // merge: one warp per query head on the tensor-core path (segments of 3 to 8 heads), one warp per segment
+  // (1 or 2 heads) on the CUDA-core path; eight warps per block
+  const int hw = uses_mma(args.group) ? 1 : args.heads_per_unit;
+  const long long warps = (long long)args.num_seqs * args.num_kv_heads * args.n_chunks * (args.heads_per_unit / hw);
+  const dim3 mgrid((unsigned)((warps + 7) / 8)), mblock(256);
+  if (hw == 2)
+    e = launch_pdl(pa::decode_merge_kernel<E, D, 2, 8>, mgrid, mblock, 0, stream, args);
+  else if (uses_mma(args.group))
+    e = launch_pdl(pa::decode_merge_kernel<E, D, 1, 4>, mgrid, mblock, 0, stream, args);
+  else
+    e = launch_pdl(pa::decode_merge_kernel<E, D, 1, 16>, mgrid, mblock, 0, stream, args);
   if (e != cudaSuccess) return record(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
@@ -488,9 +487,6 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
       (out_seq_stride % 8))
     return PA_ERR_ALIGN;
   if (!std::isfinite(scale)) return PA_ERR_SHAPE;
-  int sms = 0;
-  rc = current_sms(&sms);
-  if (rc != PA_OK) return rc;
   LaunchPlan lp;
   rc = plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, dtype, &lp);
   if (rc != PA_OK) return rc;
@@ -534,8 +530,8 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == PA_BFLOAT16;
   if (head_dim == 128)
-    return bf16 ? launch_decode_d<pa::BF16, 128>(a, lp, dtype, sms, st) : launch_decode_d<pa::F16, 128>(a, lp, dtype, sms, st);
-  return bf16 ? launch_decode_d<pa::BF16, 64>(a, lp, dtype, sms, st) : launch_decode_d<pa::F16, 64>(a, lp, dtype, sms, st);
+    return bf16 ? launch_decode_d<pa::BF16, 128>(a, lp, dtype, st) : launch_decode_d<pa::F16, 128>(a, lp, dtype, st);
+  return bf16 ? launch_decode_d<pa::BF16, 64>(a, lp, dtype, st) : launch_decode_d<pa::F16, 64>(a, lp, dtype, st);
 }
 
 int pa_get_device_status(uint32_t *status_out, int32_t clear, void *stream) {

@@ -706,9 +706,10 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
 // summed in increasing chunk order (deterministic).  Built for latency, since it runs after the split grid
 // has drained: the pieces' (m, l) and the partial rows of the first MB pieces are requested together, so a
 // segment cut into at most MB pieces costs two dependent trips to memory after the wait (tile prefix, then
-// pieces).  Blocks of two warps, so registers, not block slots, bound the warps per SM.
+// pieces).  Eight warps per block: with more, smaller blocks the grid took measurably longer to get
+// through the SMs behind the split kernel (4096 blocks of two warps: +20 us on a 256-sequence batch).
 template <class E, int D, int HW, int MB>
-__global__ void __launch_bounds__(64) decode_merge_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(256, 1) decode_merge_kernel(const DecodeArgs a) {
   static_assert(32 % MB == 0, "a batch of pieces never straddles a 32-piece window");
   constexpr int DPL = D / 32;  // dims per lane (4 or 2)
   const int lane = threadIdx.x & 31;
@@ -853,107 +854,6 @@ __global__ void __launch_bounds__(64) decode_merge_kernel(const DecodeArgs a) {
           make_uint2(E::narrow2(o[gg][0], o[gg][1]), E::narrow2(o[gg][2], o[gg][3]));
     } else {
       *reinterpret_cast<uint32_t *>(dst + gg * D) = E::narrow2(o[gg][0], o[gg][1]);
-    }
-  }
-}
-
-// Merge for the tensor-core path: one warp per (sequence, query head), eight
-// warps per block, the same arithmetic and order as decode_merge_kernel (lane
-// p holds piece p's (m, l) and weight; partial rows are loaded eight at a
-// time once the maximum is known).  Measured faster than decode_merge_kernel
-// when a segment carries 3 to 8 heads.
-template <class E, int D>
-__global__ void __launch_bounds__(256) decode_merge_heads_kernel(const DecodeArgs a) {
-  constexpr int DPL = D / 32;  // dims per lane (4 or 2)
-  const int lane = threadIdx.x & 31;
-  grid_dependency_wait();  // the split kernel's pieces and tile prefix
-  grid_launch_dependents();
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ws_queue = 0ull;  // leave the chunk counter clear
-  const int S = a.num_seqs;
-  const ChunkPlan plan = plan_chunks(a, __ldg(a.ws_tiles + S));
-  const int HC = a.num_kv_heads * a.n_chunks;
-  const int G = a.heads_per_unit;
-  const long long total = (long long)S * a.num_q_heads;
-  const long long nw = (long long)gridDim.x * (blockDim.x / 32);
-  for (long long w = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); w < total; w += nw) {
-    const int s = (int)(w / a.num_q_heads);
-    const int hq = (int)(w - (long long)s * a.num_q_heads);
-    const int L = __ldg(a.context_lens + s);
-    const int pt0 = __ldg(a.ws_tiles + s), pt1 = __ldg(a.ws_tiles + s + 1);
-    uint16_t *dst = a.out + (long long)s * a.out_seq_stride + (long long)hq * D + lane * DPL;
-    float o[DPL];
-#pragma unroll
-    for (int k = 0; k < DPL; ++k) o[k] = 0.f;
-    if (!context_ok(a, L) || L == 0) {
-      if (lane == 0 && L != 0)
-        atomicOr(&g_status, (L < 0 || (long long)L > (long long)a.table_stride * a.block_size)
-                                ? PA_DEV_ERR_CONTEXT
-                                : PA_DEV_ERR_CONTEXT_HINT);
-    } else {
-      const int h = hq / a.group;
-      const int r = hq - h * a.group;
-      const int ch = r / G;
-      const int gg = r - ch * G;
-      const int nt = pt1 - pt0;
-      const long long seg0 = (long long)pt0 * HC + (long long)(h * a.n_chunks + ch) * nt;
-      const long long c_first = plan.chunk_of(seg0), c_last = plan.chunk_of(seg0 + nt - 1);
-      if (c_first == c_last) continue;  // one chunk held the whole segment: the split kernel wrote the row
-      const int n = (int)(c_last - c_first + 1);
-      auto piece_row = [&](int p) -> int {  // partial row of piece p (chunk c_first + p)
-        const long long c = c_first + p;
-        const int slot = (p == 0 && seg0 > plan.start(c)) ? 1 : 0;
-        return (int)((c * 2 + slot) * G + gg);
-      };
-      // pass 1: maximum and validity over all pieces; lane p keeps piece p of the first 32
-      float2 ml0 = make_float2(-INFINITY, 0.f);
-      if (lane < n) ml0 = __ldg(a.ws_ml + piece_row(lane));
-      float M = ml0.x;
-      bool err = lane < n && ml0.y < 0.f;
-      for (int p = lane + 32; p < n; p += 32) {
-        const float2 ml = __ldg(a.ws_ml + piece_row(p));
-        M = fmaxf(M, ml.x);
-        err |= ml.y < 0.f;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
-      err = __any_sync(FULL, err);
-      if (!err) {
-        float l = 0.f;
-        for (int base = 0; base < n; base += 32) {
-          const int p = base + lane;
-          const float2 ml = base == 0 ? ml0 : (p < n ? __ldg(a.ws_ml + piece_row(p)) : make_float2(-INFINITY, 0.f));
-          const float wgt = p < n ? exp2f(ml.x - M) : 0.f;
-          const int row = p < n ? piece_row(p) : 0;
-          l = fmaf(ml.y, wgt, l);
-          const int cnt = min(32, n - base);
-#pragma unroll 8
-          for (int q = 0; q < cnt; ++q) {
-            const float wq = __shfl_sync(FULL, wgt, q);
-            const int rq = __shfl_sync(FULL, row, q);
-            const float *src = a.ws_acc + (long long)rq * D + lane * DPL;
-            if constexpr (DPL == 4) {
-              const float4 t = __ldg(reinterpret_cast<const float4 *>(src));
-              o[0] = fmaf(wq, t.x, o[0]);
-              o[1] = fmaf(wq, t.y, o[1]);
-              o[2] = fmaf(wq, t.z, o[2]);
-              o[3] = fmaf(wq, t.w, o[3]);
-            } else {
-              const float2 t = __ldg(reinterpret_cast<const float2 *>(src));
-              o[0] = fmaf(wq, t.x, o[0]);
-              o[1] = fmaf(wq, t.y, o[1]);
-            }
-          }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(FULL, l, off);
-#pragma unroll
-        for (int k = 0; k < DPL; ++k) o[k] = o[k] / l;
-      }
-    }
-    if constexpr (DPL == 4) {
-      *reinterpret_cast<uint2 *>(dst) = make_uint2(E::narrow2(o[0], o[1]), E::narrow2(o[2], o[3]));
-    } else {
-      *reinterpret_cast<uint32_t *>(dst) = E::narrow2(o[0], o[1]);
     }
   }
 }
