@@ -179,6 +179,11 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
  * Runs on the tensor cores (tcgen05, tensor memory accumulators): work items
  * of 256 new tokens of one query head, taken from a per-call queue by
  * persistent CTAs; computes in fp32 with P rounded to the storage type.
+ * The queue is one of 64 work counters in the library's device memory,
+ * handed to successive calls in turn and cleared on the call's stream before
+ * its launch: at most 64 calls may execute at the same time on one device
+ * (calls on one stream never overlap), and a call captured in a CUDA graph
+ * keeps the counter it was captured with.
  * Sequences with one new token cost a whole 128-row tile each here: batch
  * them through pa_decode; sequences with none cost a few microseconds per
  * thousand (query tile, head) slots of max_query_len.  Device-side errors: L_s < n_s or L_s > block_table_stride *
