@@ -84,3 +84,14 @@ def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
     assert line["value"] > 0 and line["higher_is_better"] is True and line["steps"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
+    """Under torchrun the reference arm runs on rank 0 alone; the other ranks exit 0 without work or output."""
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "tiny_decode", "--gpus", "2",
+                                      "--steps", "2", "--warmup", "1"])
+    assert bench.main() == 0
+    assert capsys.readouterr().out.strip() == ""
