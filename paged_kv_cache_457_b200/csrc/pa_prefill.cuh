@@ -83,6 +83,25 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// c + lo + hi of two packed 2-byte values, widened exactly by the mixed-precision fma (times 1.0):
+// the row sum adds the rounded P values that the PV product uses, so the weights sum to one.
+template <class E>
+__device__ __forceinline__ float add_packed(uint32_t pk, float c) {
+  float d;
+  if constexpr (std::is_same<E, BF16>::value) {
+    asm("{\n\t.reg .b16 p0, p1, one;\n\tmov.b16 one, 0x3F80;\n\tmov.b32 {p0, p1}, %1;\n\t"
+        "fma.rn.f32.bf16 %0, p0, one, %2;\n\tfma.rn.f32.bf16 %0, p1, one, %0;\n\t}"
+        : "=f"(d)
+        : "r"(pk), "f"(c));
+  } else {
+    asm("{\n\t.reg .b16 p0, p1, one;\n\tmov.b16 one, 0x3C00;\n\tmov.b32 {p0, p1}, %1;\n\t"
+        "fma.rn.f32.f16 %0, p0, one, %2;\n\tfma.rn.f32.f16 %0, p1, one, %0;\n\t}"
+        : "=f"(d)
+        : "r"(pk), "f"(c));
+  }
+  return d;
+}
+
 // All lanes wait on the same barrier phase; the warp agrees on the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
   const bool ok = mbar_wait_bounded(bar, parity, limit_ns);
@@ -503,9 +522,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             // masked scores are -inf: 2^-inf = 0
             const float p0 = ex2(fmaf(sv[c * 32 + 2 * i], a.scale_log2, -m));
             const float p1 = ex2(fmaf(sv[c * 32 + 2 * i + 1], a.scale_log2, -m));
-            sum4[(2 * i) & 3] += p0;
-            sum4[(2 * i + 1) & 3] += p1;
             pk[i] = E::narrow2(p0, p1);
+            sum4[i & 3] = add_packed<E>(pk[i], sum4[i & 3]);
           }
           tc::st16(t_s + c * 16, pk);
         }
