@@ -40,7 +40,8 @@ def from_bits(bits, dtype: str) -> np.ndarray:
     bits = np.asarray(bits, dtype=np.uint16)
     if dtype == "fp16":
         return bits.view(np.float16).astype(np.float64)
-    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # signalling-NaN patterns widen to NaN, which is the point
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def paged(logical, bs, num_blocks, rng, nan_fill=True, dtype="fp16", shared=None):
@@ -135,7 +136,8 @@ def pin_widen_bf16(lib=None):
 
 def pin_page_table_example(lib=None):
     """Section 4.2's figure: A -> physical 7,2,5; B -> two free pages; q = 0 gives plain means."""
-    g = json.load(open(GOLDEN))
+    with open(GOLDEN) as f:
+        g = json.load(f)
     bs, nb = g["block_size"], g["num_blocks"]
     u = g["uniform_attention"]
     d = u["head_dim"]

@@ -27,7 +27,8 @@ def lib():
 def declared_functions():
     names = []
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
-        text = open(h).read()
+        with open(h) as f:
+            text = f.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         names += re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)
     return sorted(set(names))

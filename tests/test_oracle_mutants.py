@@ -86,7 +86,8 @@ def mutant_results(tmp_path_factory):
     processes at a time; returns {name: failing pins}."""
     from concurrent.futures import ThreadPoolExecutor
     d = tmp_path_factory.mktemp("mutants")
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     libs = {"__control__": str(d / "lib_control.so")}
     oracle.build(SRC, libs["__control__"])
     for name, (old, new) in MUTANTS.items():
