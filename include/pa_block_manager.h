@@ -126,6 +126,30 @@ int pa_bm_build_decode_step(pa_block_manager *bm, const int64_t *seq_ids, int64_
                             int32_t *block_tables, int32_t *context_lens, int64_t *slot_mapping,
                             int64_t *copy_pairs, int64_t copy_capacity, int64_t *num_copies);
 
+/* One prefill (or chunked-prefill) step of a continuous batch: sequence i
+ * (device pool, distinct ids) brings new_tokens[i] >= 0 tokens.  Their slots
+ * are reserved as num_new successive pa_bm_append_slot calls would (a private
+ * copy of a shared, partly full last page before the first of them, a fresh
+ * page at every page boundary), then the step's arrays for pa_write_kv and
+ * pa_prefill are filled:
+ *   block_tables   int32 [num_seqs][table_stride], rows padded with -1;
+ *   query_start    int32 [num_seqs + 1], query_start[0] = 0, the new tokens'
+ *                  prefix sum (sequence i's rows of q are query_start[i] ..);
+ *   context_lens   int32 [num_seqs], tokens including the new ones;
+ *   slot_mapping   int64 [slot_capacity], the new tokens' slots in row order
+ *                  (sequence by sequence); the total must fit;
+ *   copy_pairs     int64 [copy_capacity][2], the copy-on-write pairs, in
+ *                  order; *num_copies gets their number (num_seqs pairs
+ *                  always suffice).
+ * A sequence with no new tokens gets its table and length only.  The whole
+ * step fails without change if the pool runs out, a table is longer than
+ * table_stride, a length or the token total passes int32, or an output array
+ * is too small. */
+int pa_bm_build_prefill_step(pa_block_manager *bm, const int64_t *seq_ids, const int64_t *new_tokens,
+                             int64_t num_seqs, int64_t table_stride, int32_t *block_tables, int32_t *query_start,
+                             int32_t *context_lens, int64_t *slot_mapping, int64_t slot_capacity,
+                             int64_t *copy_pairs, int64_t copy_capacity, int64_t *num_copies);
+
 /* Moves num_seqs device-pool sequences to the host pool (preemption).
  * mapping int64 [capacity][2] gets the (device page, host page) pairs to
  * copy with pa_swap_blocks (device pools as source, host pools as

@@ -27,7 +27,7 @@ __all__ = [
     "PagedAttentionError", "write_kv", "decode", "decode_workspace_size", "copy_blocks", "swap_blocks", "prefill",
     "device_status", "launch_count", "debug_wait_timeout", "library_path", "load_library", "EXPORTED_SYMBOLS",
     "DEV_ERR_BLOCK_ID", "DEV_ERR_CONTEXT", "DEV_ERR_CONTEXT_HINT", "DEV_ERR_SLOT", "DEV_ERR_TIMEOUT",
-    "BlockManager", "BlockManagerError", "DecodeStepPlan",
+    "BlockManager", "BlockManagerError", "DecodeStepPlan", "PrefillStepPlan",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -49,7 +49,7 @@ EXPORTED_SYMBOLS = (
     "pa_debug_wait_timeout", "pa_version", "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_device_blocks", "pa_bm_num_free_host_blocks",
     "pa_bm_ref_count", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_num_tokens",
-    "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step",
+    "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step", "pa_bm_build_prefill_step",
     "pa_bm_swap_out", "pa_bm_swap_in", "pa_prefill",
 )
 
@@ -320,4 +320,4 @@ def debug_wait_timeout(limit_ns: int = 10_000_000) -> None:
     _check(load_library().pa_debug_wait_timeout(int(limit_ns), _stream(dev)), "pa_debug_wait_timeout")
 
 
-from .block_manager import BlockManager, BlockManagerError, DecodeStepPlan  # noqa: E402
+from .block_manager import BlockManager, BlockManagerError, DecodeStepPlan, PrefillStepPlan  # noqa: E402

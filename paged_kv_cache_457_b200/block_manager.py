@@ -45,6 +45,7 @@ def bind(lib: ctypes.CDLL) -> None:
         "pa_bm_slots": (ctypes.c_int, [vp, i64, i64, i64, vp]),
         "pa_bm_append_slot": (ctypes.c_int, [vp, i64, p64, p64, p64]),
         "pa_bm_build_decode_step": (ctypes.c_int, [vp, vp, i64, i64, vp, vp, vp, vp, i64, p64]),
+        "pa_bm_build_prefill_step": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, vp, vp, vp, i64, vp, i64, p64]),
         "pa_bm_swap_out": (ctypes.c_int, [vp, vp, i64, vp, i64, p64]),
         "pa_bm_swap_in": (ctypes.c_int, [vp, vp, i64, vp, i64, p64]),
     }
@@ -60,6 +61,16 @@ class DecodeStepPlan:
     block_tables: np.ndarray   # int32 [S, table_stride], -1 padded
     context_lens: np.ndarray   # int32 [S], including the new token
     slot_mapping: np.ndarray   # int64 [S], the new token's slot
+    copy_pairs: np.ndarray     # int64 [n, 2], copy-on-write pairs to apply first
+
+
+@dataclass
+class PrefillStepPlan:
+    """Host arrays of one prefill (or chunked-prefill) step, as pa_write_kv and pa_prefill take them."""
+    block_tables: np.ndarray   # int32 [S, table_stride], -1 padded
+    query_start: np.ndarray    # int32 [S + 1], prefix sum of the new tokens
+    context_lens: np.ndarray   # int32 [S], including the new tokens
+    slot_mapping: np.ndarray   # int64 [total new tokens], row order
     copy_pairs: np.ndarray     # int64 [n, 2], copy-on-write pairs to apply first
 
 
@@ -158,6 +169,25 @@ class BlockManager:
                                                       _p(slots), _p(pairs), S, ctypes.byref(n)),
                     "pa_bm_build_decode_step")
         return DecodeStepPlan(tables, lens, slots, pairs[: n.value].copy())
+
+    def build_prefill_step(self, seq_ids, new_tokens, table_stride: int) -> PrefillStepPlan:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n_new = np.ascontiguousarray(new_tokens, dtype=np.int64)
+        S = len(ids)
+        if len(n_new) != S:
+            raise BlockManagerError(-20, "pa_bm_build_prefill_step")
+        total = int(n_new.sum()) if S else 0
+        tables = np.empty((S, int(table_stride)), dtype=np.int32)
+        qs = np.empty(S + 1, dtype=np.int32)
+        lens = np.empty(S, dtype=np.int32)
+        slots = np.empty(max(total, 0), dtype=np.int64)
+        pairs = np.empty((S, 2), dtype=np.int64)
+        n = ctypes.c_int64(0)
+        self._check(self._lib.pa_bm_build_prefill_step(self._h, _p(ids), _p(n_new), S, int(table_stride), _p(tables),
+                                                       _p(qs), _p(lens), _p(slots), slots.size, _p(pairs), S,
+                                                       ctypes.byref(n)),
+                    "pa_bm_build_prefill_step")
+        return PrefillStepPlan(tables, qs, lens, slots, pairs[: n.value].copy())
 
     def _move(self, fn, seq_ids, what):
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)

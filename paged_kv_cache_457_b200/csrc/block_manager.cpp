@@ -348,6 +348,77 @@ int pa_bm_build_decode_step(pa_block_manager *bm, const int64_t *seq_ids, int64_
   });
 }
 
+int pa_bm_build_prefill_step(pa_block_manager *bm, const int64_t *seq_ids, const int64_t *new_tokens,
+                             int64_t num_seqs, int64_t table_stride, int32_t *block_tables, int32_t *query_start,
+                             int32_t *context_lens, int64_t *slot_mapping, int64_t slot_capacity,
+                             int64_t *copy_pairs, int64_t copy_capacity, int64_t *num_copies) {
+  return guarded(bm, [&] {
+    if (num_seqs < 0 || table_stride < 0 || slot_capacity < 0 || copy_capacity < 0 || !num_copies || !query_start)
+      return PA_BM_ERR_ARG;
+    if (num_seqs > 0 && (!seq_ids || !new_tokens || !context_lens || (table_stride > 0 && !block_tables)))
+      return PA_BM_ERR_ARG;
+    // Plan: pages and copies the appends will take, simulating the references
+    // that earlier copies of this step drop from shared last pages.
+    std::vector<pa_block_manager::Seq *> list;
+    list.reserve(static_cast<size_t>(num_seqs));
+    std::unordered_set<int64_t> seen;
+    std::unordered_map<int32_t, int32_t> dropped;
+    int64_t pages = 0, copies = 0, total = 0;
+    const int64_t int32_max = std::numeric_limits<int32_t>::max();
+    for (int64_t i = 0; i < num_seqs; ++i) {
+      auto it = bm->seqs.find(seq_ids[i]);
+      if (it == bm->seqs.end()) return PA_BM_ERR_UNKNOWN;
+      auto &s = it->second;
+      if (s.host) return PA_BM_ERR_STATE;
+      if (!seen.insert(seq_ids[i]).second) return PA_BM_ERR_ARG;
+      const int64_t n = new_tokens[i];
+      if (n < 0 || n > int32_max - s.tokens || n > int32_max - total) return PA_BM_ERR_ARG;
+      total += n;
+      if (n > 0) {
+        const bool fresh_row = s.tokens % bm->block_size == 0;
+        if (!fresh_row && bm->append_needs_page(s, dropped[s.table.back()])) {  // private copy of the last page
+          ++pages;
+          ++copies;
+          ++dropped[s.table.back()];
+        }
+        pages += bm->pages_for(s.tokens + n) - bm->pages_for(s.tokens);
+      }
+      if (bm->pages_for(s.tokens + n) > table_stride) return PA_BM_ERR_CAPACITY;
+      list.push_back(&s);
+    }
+    *num_copies = copies;
+    if (pages > bm->dev.num_free()) return PA_BM_ERR_NO_SPACE;
+    if (total > slot_capacity || (total > 0 && !slot_mapping)) return PA_BM_ERR_CAPACITY;
+    if (copies > copy_capacity || (copies > 0 && !copy_pairs)) return PA_BM_ERR_CAPACITY;
+    for (int64_t i = 0; i < num_seqs; ++i) {
+      auto *s = list[static_cast<size_t>(i)];
+      s->table.reserve(static_cast<size_t>(bm->pages_for(s->tokens + new_tokens[i])));
+    }
+    // Mutation: cannot fail from here on.
+    int64_t c = 0, row = 0;
+    query_start[0] = 0;
+    for (int64_t i = 0; i < num_seqs; ++i) {
+      auto &s = *list[static_cast<size_t>(i)];
+      for (int64_t k = 0; k < new_tokens[i]; ++k, ++row) {
+        int64_t src, dst;
+        bm->append(s, &slot_mapping[row], &src, &dst);
+        if (src >= 0) {
+          copy_pairs[2 * c] = src;
+          copy_pairs[2 * c + 1] = dst;
+          ++c;
+        }
+      }
+      query_start[i + 1] = static_cast<int32_t>(row);
+      context_lens[i] = static_cast<int32_t>(s.tokens);
+      int32_t *trow = block_tables + i * table_stride;
+      const int64_t nb = static_cast<int64_t>(s.table.size());
+      std::copy(s.table.begin(), s.table.end(), trow);
+      std::fill(trow + nb, trow + table_stride, -1);
+    }
+    return PA_BM_OK;
+  });
+}
+
 int pa_bm_swap_out(pa_block_manager *bm, const int64_t *seq_ids, int64_t num_seqs, int64_t *mapping,
                    int64_t capacity, int64_t *num_pairs) {
   return guarded(bm, [&] { return bm->move(seq_ids, num_seqs, true, mapping, capacity, num_pairs); });

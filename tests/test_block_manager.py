@@ -375,3 +375,120 @@ def test_concurrent_calls_keep_the_pool_consistent():
             np.add.at(refs, t, 1)
     assert [bm.ref_count(b) for b in range(4096)] == refs.tolist()
     assert bm.num_free_device_blocks == int((refs == 0).sum())
+
+
+def test_prefill_step_reserves_a_chunk_per_sequence():
+    """A chunk of new tokens per sequence: slots continue each sequence, pages are taken at page
+    boundaries, query_start is the prefix sum, and a sequence with no new tokens keeps its state."""
+    bm = pa.BlockManager(16, 64, 0)
+    bm.add_sequence(0, 100)   # 7 pages, 4 rows used in the last
+    bm.add_sequence(1, 32)    # 2 full pages
+    bm.add_sequence(2, 5)
+    free0 = bm.num_free_device_blocks
+    plan = bm.build_prefill_step([0, 1, 2], [50, 1, 0], 12)
+    assert isinstance(plan, pa.PrefillStepPlan)
+    assert plan.query_start.tolist() == [0, 50, 51, 51]
+    assert plan.context_lens.tolist() == [150, 33, 5]
+    assert len(plan.slot_mapping) == 51 and len(plan.copy_pairs) == 0
+    assert np.array_equal(plan.slot_mapping[:50], bm.slots(0, 100, 50))
+    assert plan.slot_mapping[50] == bm.slots(1, 32, 1)[0]
+    assert bm.num_free_device_blocks == free0 - (3 + 1)   # pages 8-10 of sequence 0, page 3 of sequence 1
+    for i, sid in enumerate([0, 1, 2]):
+        t = bm.block_table(sid)
+        assert np.array_equal(plan.block_tables[i, :len(t)], t) and np.all(plan.block_tables[i, len(t):] == -1)
+
+
+def test_prefill_step_copies_a_shared_partial_page_once():
+    """Two sequences share a partly full last page: the first to append gets a private copy, after
+    which the second is the page's only owner and appends in place."""
+    bm = pa.BlockManager(16, 32, 0)
+    bm.add_sequence(0, 37)
+    bm.fork(0, 1)
+    last = int(bm.block_table(0)[-1])
+    assert bm.ref_count(last) == 2
+    plan = bm.build_prefill_step([0, 1], [20, 3], 8)
+    assert plan.copy_pairs.shape == (1, 2) and plan.copy_pairs[0, 0] == last
+    assert int(bm.block_table(0)[2]) == plan.copy_pairs[0, 1]
+    assert int(bm.block_table(1)[2]) == last and bm.ref_count(last) == 1
+    assert plan.context_lens.tolist() == [57, 40]
+
+
+def test_prefill_step_is_all_or_nothing():
+    bm = pa.BlockManager(16, 6, 0)
+    bm.add_sequence(0, 20)
+    bm.add_sequence(1, 30)
+    before = (bm.num_free_device_blocks, bm.block_table(0).tolist(), bm.block_table(1).tolist(),
+              bm.num_tokens(0), bm.num_tokens(1))
+
+    def state():
+        return (bm.num_free_device_blocks, bm.block_table(0).tolist(), bm.block_table(1).tolist(),
+                bm.num_tokens(0), bm.num_tokens(1))
+
+    with pytest.raises(pa.BlockManagerError) as e:   # 2 + 1 pages needed, 2 free
+        bm.build_prefill_step([0, 1], [40, 20], 8)
+    assert e.value.code == -21 and state() == before
+    with pytest.raises(pa.BlockManagerError) as e:   # the table of sequence 0 would need 3 entries
+        bm.build_prefill_step([0, 1], [20, 1], 2)
+    assert e.value.code == -25 and state() == before
+    for bad in ([0, 0], [0, 99]):
+        with pytest.raises(pa.BlockManagerError):
+            bm.build_prefill_step(bad, [1, 1], 8)
+        assert state() == before
+    with pytest.raises(pa.BlockManagerError):
+        bm.build_prefill_step([0, 1], [1, -1], 8)
+    with pytest.raises(pa.BlockManagerError):
+        bm.build_prefill_step([0, 1], [1], 8)
+    assert state() == before
+
+
+def test_manager_plans_through_the_oracle_prefill():
+    """Chunked prefill steps planned by the manager (forked sequences, ragged chunks, idle
+    sequences), applied with the oracle's copy and write, give the same causal attention as the
+    oracle over each sequence's tokens laid out contiguously."""
+    rng = np.random.default_rng(5)
+    dtype, hkv, hq, d, bs, nb = "bf16", 2, 4, 64, 16, 64
+    from oracle_pins import to_bits
+    bm = pa.BlockManager(bs, nb, 0)
+    kc = np.zeros((nb, hkv, bs, d), dtype=np.uint16)
+    vc = np.zeros_like(kc)
+    logical = {}
+    for sid, n in ((0, 29), (1, 16)):
+        bm.add_sequence(sid, n)
+        k = to_bits(rng.standard_normal((n, hkv, d)), dtype)
+        v = to_bits(rng.standard_normal((n, hkv, d)), dtype)
+        kc, vc = oracle.write_kv(k, v, kc, vc, bm.slots(sid, 0, n), bs)
+        logical[sid] = (k, v)
+    bm.fork(0, 2)
+    logical[2] = logical[0]
+    ids = [0, 1, 2]
+    for step in range(6):
+        chunk = [int(x) for x in rng.integers(0, 40, size=len(ids))]
+        plan = bm.build_prefill_step(ids, chunk, 16)
+        if len(plan.copy_pairs):
+            kc, vc = oracle.copy_blocks(kc, vc, kc, vc, plan.copy_pairs)
+        total = int(sum(chunk))
+        k = to_bits(rng.standard_normal((total, hkv, d)), dtype)
+        v = to_bits(rng.standard_normal((total, hkv, d)), dtype)
+        kc, vc = oracle.write_kv(k, v, kc, vc, plan.slot_mapping, bs)
+        for i, sid in enumerate(ids):
+            a, b = plan.query_start[i], plan.query_start[i + 1]
+            lk, lv = logical[sid]
+            logical[sid] = (np.concatenate([lk, k[a:b]]), np.concatenate([lv, v[a:b]]))
+        q = to_bits(rng.standard_normal((total, hq, d)), dtype)
+        got = oracle.prefill(q, kc, vc, plan.block_tables, plan.query_start, plan.context_lens, 0.125, dtype)
+        for i, sid in enumerate(ids):
+            a, b = int(plan.query_start[i]), int(plan.query_start[i + 1])
+            if a == b:
+                continue
+            lk, lv = logical[sid]
+            L = len(lk)
+            assert L == plan.context_lens[i]
+            nblk = -(-L // bs)
+            ck = np.zeros((nblk, hkv, bs, d), dtype=np.uint16)
+            cv = np.zeros_like(ck)
+            for j in range(L):
+                ck[j // bs, :, j % bs] = lk[j]
+                cv[j // bs, :, j % bs] = lv[j]
+            want = oracle.prefill(q[a:b], ck, cv, np.arange(nblk, dtype=np.int32)[None], np.array([0, b - a], np.int32),
+                                  np.array([L], np.int32), 0.125, dtype)
+            assert np.array_equal(got[a:b], want), f"step {step} sequence {sid}"
