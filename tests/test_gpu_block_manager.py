@@ -93,3 +93,59 @@ def test_manager_driven_steps_match_oracle(dtype, hq, hkv, d, bs):
     for sid in list(logical):
         bm.free_sequence(sid)
     assert bm.num_free_device_blocks == nb and bm.num_free_host_blocks == nh
+
+
+def test_manager_driven_chunked_prefill_matches_oracle():
+    """Chunked prefill steps planned by the native pool (a forked pair sharing a partly full page,
+    ragged chunks, idle sequences) through copy_blocks, write_kv and the tensor-core prefill, each
+    sequence's rows compared with the oracle over its own tokens laid out contiguously."""
+    require_gpu()
+    dtype, hq, hkv, d, bs = "fp16", 8, 2, 128, 16
+    rng = np.random.default_rng(17)
+    nb = 64
+    bm = pa.BlockManager(bs, nb, 0)
+    tdt = TORCH_DT[dtype]
+    kc = torch.zeros((nb, hkv, bs, d), dtype=tdt, device="cuda")
+    vc = torch.zeros_like(kc)
+    logical = {}
+    for sid, n in ((0, 29), (1, 16)):
+        bm.add_sequence(sid, n)
+        k = to_bits(rng.standard_normal((n, hkv, d)), dtype)
+        v = to_bits(rng.standard_normal((n, hkv, d)), dtype)
+        pa.write_kv(to_dev(k, dtype), to_dev(v, dtype), kc, vc, to_dev_index(bm.slots(sid, 0, n)))
+        logical[sid] = (k, v)
+    bm.fork(0, 2)
+    logical[2] = logical[0]
+    ids = [0, 1, 2]
+    scale = 1.0 / np.sqrt(d)
+    copies = 0
+    for step in range(5):
+        chunk = [int(rng.integers(1, 40))] + [int(x) for x in rng.integers(0, 40, size=len(ids) - 1)]
+        plan = bm.build_prefill_step(ids, chunk, 16)
+        if len(plan.copy_pairs):
+            copies += len(plan.copy_pairs)
+            pa.copy_blocks(kc, vc, to_dev_index(plan.copy_pairs))
+        total = int(sum(chunk))
+        k = to_bits(rng.standard_normal((total, hkv, d)), dtype)
+        v = to_bits(rng.standard_normal((total, hkv, d)), dtype)
+        pa.write_kv(to_dev(k, dtype), to_dev(v, dtype), kc, vc, to_dev_index(plan.slot_mapping))
+        for i, sid in enumerate(ids):
+            a, b = int(plan.query_start[i]), int(plan.query_start[i + 1])
+            lk, lv = logical[sid]
+            logical[sid] = (np.concatenate([lk, k[a:b]]), np.concatenate([lv, v[a:b]]))
+        q = to_bits(rng.standard_normal((total, hq, d)), dtype)
+        out_bits = host_bits(pa.prefill(to_dev(q, dtype), kc, vc, to_dev_index(plan.block_tables),
+                                        to_dev_index(plan.query_start), to_dev_index(plan.context_lens), scale,
+                                        max(chunk)))
+        for i, sid in enumerate(ids):
+            a, b = int(plan.query_start[i]), int(plan.query_start[i + 1])
+            if a == b:
+                continue
+            ck, cv = _contiguous(*logical[sid], bs)
+            L = len(logical[sid][0])
+            ref = oracle.prefill(q[a:b], ck, cv, np.arange(len(ck), dtype=np.int32)[None],
+                                 np.array([0, b - a], np.int32), np.array([L], np.int32), scale, dtype)
+            compare(out_bits[a:b], ref, dtype, what=f"step {step} sequence {sid}")
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+    assert copies >= 1  # the first of the forked pair to append split the shared partial page
