@@ -150,6 +150,15 @@ int pa_bm_build_prefill_step(pa_block_manager *bm, const int64_t *seq_ids, const
                              int32_t *context_lens, int64_t *slot_mapping, int64_t slot_capacity,
                              int64_t *copy_pairs, int64_t copy_capacity, int64_t *num_copies);
 
+/* What a step would take, without taking it: sequence i (device pool,
+ * distinct ids) brings new_tokens[i] >= 0 tokens (1 each for a decode step).
+ * *pages gets the fresh device pages the step needs (copy-on-write copies
+ * included), *copies the copy-on-write pairs it would produce.  Compare with
+ * pa_bm_num_free_device_blocks to decide admission or preemption before
+ * building the step. */
+int pa_bm_step_needs(const pa_block_manager *bm, const int64_t *seq_ids, const int64_t *new_tokens, int64_t num_seqs,
+                     int64_t *pages, int64_t *copies);
+
 /* Moves num_seqs device-pool sequences to the host pool (preemption).
  * mapping int64 [capacity][2] gets the (device page, host page) pairs to
  * copy with pa_swap_blocks (device pools as source, host pools as

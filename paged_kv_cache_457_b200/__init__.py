@@ -49,7 +49,7 @@ EXPORTED_SYMBOLS = (
     "pa_debug_wait_timeout", "pa_version", "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_device_blocks", "pa_bm_num_free_host_blocks",
     "pa_bm_ref_count", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_num_tokens",
-    "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step", "pa_bm_build_prefill_step",
+    "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step", "pa_bm_build_prefill_step", "pa_bm_step_needs",
     "pa_bm_swap_out", "pa_bm_swap_in", "pa_prefill",
 )
 

@@ -46,6 +46,7 @@ def bind(lib: ctypes.CDLL) -> None:
         "pa_bm_append_slot": (ctypes.c_int, [vp, i64, p64, p64, p64]),
         "pa_bm_build_decode_step": (ctypes.c_int, [vp, vp, i64, i64, vp, vp, vp, vp, i64, p64]),
         "pa_bm_build_prefill_step": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, vp, vp, vp, i64, vp, i64, p64]),
+        "pa_bm_step_needs": (ctypes.c_int, [vp, vp, vp, i64, p64, p64]),
         "pa_bm_swap_out": (ctypes.c_int, [vp, vp, i64, vp, i64, p64]),
         "pa_bm_swap_in": (ctypes.c_int, [vp, vp, i64, vp, i64, p64]),
     }
@@ -188,6 +189,17 @@ class BlockManager:
                                                        ctypes.byref(n)),
                     "pa_bm_build_prefill_step")
         return PrefillStepPlan(tables, qs, lens, slots, pairs[: n.value].copy())
+
+    def step_needs(self, seq_ids, new_tokens) -> tuple:
+        """(fresh device pages, copy-on-write pairs) a step would take; nothing changes."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n_new = np.ascontiguousarray(new_tokens, dtype=np.int64)
+        if len(n_new) != len(ids):
+            raise BlockManagerError(-20, "pa_bm_step_needs")
+        pages, copies = ctypes.c_int64(0), ctypes.c_int64(0)
+        self._check(self._lib.pa_bm_step_needs(self._h, _p(ids), _p(n_new), len(ids), ctypes.byref(pages),
+                                               ctypes.byref(copies)), "pa_bm_step_needs")
+        return pages.value, copies.value
 
     def _move(self, fn, seq_ids, what):
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)

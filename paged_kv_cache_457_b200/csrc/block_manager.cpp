@@ -86,6 +86,41 @@ struct pa_block_manager {
     ++s.tokens;
   }
 
+  // Plan of a step in which sequence i brings new_tokens[i] >= 0 tokens: the fresh device pages and the
+  // copy-on-write pairs its appends will take (simulating the references that earlier copies of the same
+  // step drop from shared last pages), the token total, and the sequences in order.  Tables longer than
+  // table_stride fail with PA_BM_ERR_CAPACITY.  Changes nothing.
+  int plan_step(const int64_t *ids, const int64_t *new_tokens, int64_t n, int64_t table_stride, int64_t *pages,
+                int64_t *copies, int64_t *total, std::vector<Seq *> *list) {
+    list->reserve(static_cast<size_t>(n));
+    std::unordered_set<int64_t> seen;
+    std::unordered_map<int32_t, int32_t> dropped;
+    const int64_t int32_max = std::numeric_limits<int32_t>::max();
+    *pages = *copies = *total = 0;
+    for (int64_t i = 0; i < n; ++i) {
+      auto it = seqs.find(ids[i]);
+      if (it == seqs.end()) return PA_BM_ERR_UNKNOWN;
+      auto &s = it->second;
+      if (s.host) return PA_BM_ERR_STATE;
+      if (!seen.insert(ids[i]).second) return PA_BM_ERR_ARG;
+      const int64_t add = new_tokens[i];
+      if (add < 0 || add > int32_max - s.tokens || add > int32_max - *total) return PA_BM_ERR_ARG;
+      *total += add;
+      if (add > 0) {
+        const bool fresh_row = s.tokens % block_size == 0;
+        if (!fresh_row && append_needs_page(s, dropped[s.table.back()])) {  // private copy of the last page
+          ++*pages;
+          ++*copies;
+          ++dropped[s.table.back()];
+        }
+        *pages += pages_for(s.tokens + add) - pages_for(s.tokens);
+      }
+      if (pages_for(s.tokens + add) > table_stride) return PA_BM_ERR_CAPACITY;
+      list->push_back(&s);
+    }
+    return PA_BM_OK;
+  }
+
   // Moves whole sequences from pool `from` to pool `to` (see swap_out / swap_in).
   int move(const int64_t *ids, int64_t n, bool to_host, int64_t *mapping, int64_t capacity, int64_t *num_pairs) {
     if (n < 0 || (n > 0 && !ids) || !num_pairs || capacity < 0 || (capacity > 0 && !mapping)) return PA_BM_ERR_ARG;
@@ -357,35 +392,10 @@ int pa_bm_build_prefill_step(pa_block_manager *bm, const int64_t *seq_ids, const
       return PA_BM_ERR_ARG;
     if (num_seqs > 0 && (!seq_ids || !new_tokens || !context_lens || (table_stride > 0 && !block_tables)))
       return PA_BM_ERR_ARG;
-    // Plan: pages and copies the appends will take, simulating the references
-    // that earlier copies of this step drop from shared last pages.
     std::vector<pa_block_manager::Seq *> list;
-    list.reserve(static_cast<size_t>(num_seqs));
-    std::unordered_set<int64_t> seen;
-    std::unordered_map<int32_t, int32_t> dropped;
     int64_t pages = 0, copies = 0, total = 0;
-    const int64_t int32_max = std::numeric_limits<int32_t>::max();
-    for (int64_t i = 0; i < num_seqs; ++i) {
-      auto it = bm->seqs.find(seq_ids[i]);
-      if (it == bm->seqs.end()) return PA_BM_ERR_UNKNOWN;
-      auto &s = it->second;
-      if (s.host) return PA_BM_ERR_STATE;
-      if (!seen.insert(seq_ids[i]).second) return PA_BM_ERR_ARG;
-      const int64_t n = new_tokens[i];
-      if (n < 0 || n > int32_max - s.tokens || n > int32_max - total) return PA_BM_ERR_ARG;
-      total += n;
-      if (n > 0) {
-        const bool fresh_row = s.tokens % bm->block_size == 0;
-        if (!fresh_row && bm->append_needs_page(s, dropped[s.table.back()])) {  // private copy of the last page
-          ++pages;
-          ++copies;
-          ++dropped[s.table.back()];
-        }
-        pages += bm->pages_for(s.tokens + n) - bm->pages_for(s.tokens);
-      }
-      if (bm->pages_for(s.tokens + n) > table_stride) return PA_BM_ERR_CAPACITY;
-      list.push_back(&s);
-    }
+    const int rc = bm->plan_step(seq_ids, new_tokens, num_seqs, table_stride, &pages, &copies, &total, &list);
+    if (rc != PA_BM_OK) return rc;
     *num_copies = copies;
     if (pages > bm->dev.num_free()) return PA_BM_ERR_NO_SPACE;
     if (total > slot_capacity || (total > 0 && !slot_mapping)) return PA_BM_ERR_CAPACITY;
@@ -417,6 +427,23 @@ int pa_bm_build_prefill_step(pa_block_manager *bm, const int64_t *seq_ids, const
     }
     return PA_BM_OK;
   });
+}
+
+int pa_bm_step_needs(const pa_block_manager *bm, const int64_t *seq_ids, const int64_t *new_tokens, int64_t num_seqs,
+                     int64_t *pages, int64_t *copies) {
+  if (!bm) return PA_BM_ERR_ARG;
+  try {
+    std::lock_guard<std::mutex> g(bm->mu);
+    if (num_seqs < 0 || !pages || !copies || (num_seqs > 0 && (!seq_ids || !new_tokens))) return PA_BM_ERR_ARG;
+    std::vector<pa_block_manager::Seq *> list;
+    int64_t total = 0;
+    // plan_step reads the state only; the cast lets it hand back the sequences it planned for
+    return const_cast<pa_block_manager *>(bm)->plan_step(seq_ids, new_tokens, num_seqs,
+                                                          std::numeric_limits<int64_t>::max(), pages, copies,
+                                                          &total, &list);
+  } catch (const std::bad_alloc &) {
+    return PA_BM_ERR_HOST_MEMORY;
+  }
 }
 
 int pa_bm_swap_out(pa_block_manager *bm, const int64_t *seq_ids, int64_t num_seqs, int64_t *mapping,

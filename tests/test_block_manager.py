@@ -492,3 +492,29 @@ def test_manager_plans_through_the_oracle_prefill():
             want = oracle.prefill(q[a:b], ck, cv, np.arange(nblk, dtype=np.int32)[None], np.array([0, b - a], np.int32),
                                   np.array([L], np.int32), 0.125, dtype)
             assert np.array_equal(got[a:b], want), f"step {step} sequence {sid}"
+
+
+def test_step_needs_predicts_every_step_without_changing_anything():
+    """step_needs gives the pages and copies that the next step then takes, for prefill chunks and
+    decode steps over forked sequences, and leaves the pool as it was."""
+    rng = np.random.default_rng(9)
+    bm = pa.BlockManager(16, 200, 0)
+    bm.add_sequence(0, 37)
+    bm.add_sequence(1, 48)
+    bm.fork(0, 2)
+    bm.fork(2, 3)
+    ids = [0, 1, 2, 3]
+    for step in range(30):
+        decode = step % 3 == 2
+        chunk = [1] * len(ids) if decode else [int(x) for x in rng.integers(0, 30, size=len(ids))]
+        tables = [bm.block_table(i).tolist() for i in ids]
+        free = bm.num_free_device_blocks
+        pages, copies = bm.step_needs(ids, chunk)
+        assert bm.num_free_device_blocks == free and [bm.block_table(i).tolist() for i in ids] == tables
+        plan = bm.build_decode_step(ids, 64) if decode else bm.build_prefill_step(ids, chunk, 64)
+        assert free - bm.num_free_device_blocks == pages, f"step {step}"
+        assert len(plan.copy_pairs) == copies, f"step {step}"
+    with pytest.raises(pa.BlockManagerError):
+        bm.step_needs([0, 0], [1, 1])
+    with pytest.raises(pa.BlockManagerError):
+        bm.step_needs([0, 7], [1, 1])
