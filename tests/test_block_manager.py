@@ -331,7 +331,7 @@ def test_manager_plans_through_the_oracle_decode():
 
 def test_concurrent_calls_keep_the_pool_consistent():
     """Calls on one manager from several host threads are serialised: after a storm of adds, forks,
-    appends and frees the reference counts still equal the tables that name each page."""
+    appends, prefill chunks and frees the reference counts still equal the tables that name each page."""
     import threading
     bm = pa.BlockManager(16, 4096)
     errors = []
@@ -349,8 +349,13 @@ def test_concurrent_calls_keep_the_pool_consistent():
                 elif r < 0.6:
                     bm.fork(int(rng.choice(mine)), sid)
                     mine.append(sid)
-                elif r < 0.85:
+                elif r < 0.75:
                     bm.append_slot(int(rng.choice(mine)))
+                elif r < 0.85:  # a chunk for a few of this thread's sequences
+                    pick = [int(x) for x in rng.choice(mine, size=min(3, len(mine)), replace=False)]
+                    chunk = [int(x) for x in rng.integers(0, 40, size=len(pick))]
+                    bm.step_needs(pick, chunk)
+                    bm.build_prefill_step(pick, chunk, 256)
                 else:
                     victim = int(rng.choice(mine))
                     bm.free_sequence(victim)
