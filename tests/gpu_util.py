@@ -10,9 +10,11 @@ from oracle_pins import from_bits, to_bits
 
 TORCH_DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
 
-# Tolerances on the attention output (fp16/bf16 storage, fp32 accumulation):
-# max |gpu - exact| <= 1e-2 over all elements, and mean |gpu - exact rounded
-# once to the output's storage type| <= 1e-3.
+# Tolerances on the attention output (fp16/bf16 storage, fp32 accumulation),
+# both against the exact fp64 oracle value: max |gpu - exact| <= 1e-2 over all
+# elements and mean |gpu - exact| <= 1e-3.  As an extra diagnostic the mean
+# distance to the exact value rounded once to the output's storage type is
+# held to the same 1e-3 (it isolates the kernel's own error from the format's).
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 
@@ -76,6 +78,9 @@ def compare(out_bits: np.ndarray, ref: np.ndarray, dtype: str, max_abs=MAX_ABS, 
     stats = {"max_abs": float(err.max(initial=0.0)), "mean_abs": float(err.mean()) if err.size else 0.0,
              "mean_abs_vs_rounded": float(err_r.mean()) if err_r.size else 0.0,
              "max_abs_vs_rounded": float(err_r.max(initial=0.0))}
+    print(f"[parity] {what}: max_abs {stats['max_abs']:.3e} mean_abs {stats['mean_abs']:.3e} "
+          f"mean_abs_vs_rounded {stats['mean_abs_vs_rounded']:.3e}")
     assert stats["max_abs"] <= max_abs, f"{what}: {stats}"
+    assert stats["mean_abs"] <= mean_abs, f"{what}: {stats}"
     assert stats["mean_abs_vs_rounded"] <= mean_abs, f"{what}: {stats}"
     return stats
