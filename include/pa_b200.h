@@ -71,6 +71,10 @@ extern "C" {
 #define PA_DEV_ERR_CONTEXT_HINT 0x4u /* context_len > the max_context_len the call was given */
 #define PA_DEV_ERR_SLOT 0x8u        /* a slot_mapping entry >= num_blocks * block_size */
 #define PA_DEV_ERR_TIMEOUT 0x10u    /* a bounded wait on a bulk copy ran out */
+#define PA_DEV_ERR_INTERNAL 0x20u   /* debug builds only: an internal index check failed; that access was skipped */
+
+/* ---- build flags (pa_build_flags) ---- */
+#define PA_BUILD_DEBUG 0x1u /* built with PA_DEBUG: every derived index is checked on the device before use */
 
 typedef enum { PA_FLOAT16 = 1, PA_BFLOAT16 = 2 } pa_dtype;
 
@@ -295,6 +299,29 @@ int pa_decode_static_workspace(const void *q, const void *k_cache, const void *v
                                int32_t block_size, int64_t num_blocks, int32_t block_table_stride,
                                int32_t max_context_len, int64_t q_seq_stride, int64_t out_seq_stride,
                                int32_t partition_tokens, int32_t dtype, void *stream);
+
+/*
+ * pa_read_bandwidth_probe -- reads `bytes` bytes at `src` (device memory,
+ * 16-byte aligned, bytes a multiple of 16) once, with every SM streaming
+ * 16-byte loads that bypass L1, and folds them into *sink (one device word,
+ * XOR-accumulated; its value means nothing).  A measurement aid with no
+ * counterpart on the pages: timed with events around it over a buffer much
+ * larger than L2, it gives the read-only HBM rate against which the decode
+ * kernels (which read K/V and write almost nothing) are best compared.
+ * bytes == 0 launches nothing.
+ */
+int pa_read_bandwidth_probe(const void *src, int64_t bytes, uint32_t *sink, void *stream);
+
+/*
+ * pa_build_flags -- PA_BUILD_* bits of this build.  A PA_DEBUG build
+ * (libpa_b200_debug.so) checks, before each access, every index the kernels
+ * derive rather than read (the tile a stream position maps to, table-window
+ * entries, cache rows, chunk and piece rows of the workspace, output rows,
+ * prefill items); a failed check skips the access and sets
+ * PA_DEV_ERR_INTERNAL.  Results are otherwise the same as the release
+ * build's.  It stands in for a memory checker on small cases.
+ */
+uint32_t pa_build_flags(void);
 
 /* pa_version -- library ABI version (major * 10000 + minor * 100 + patch). */
 int32_t pa_version(void);

@@ -25,8 +25,9 @@ import torch
 
 __all__ = [
     "PagedAttentionError", "write_kv", "decode", "decode_workspace_size", "copy_blocks", "swap_blocks", "prefill",
-    "device_status", "launch_count", "debug_wait_timeout", "library_path", "load_library", "EXPORTED_SYMBOLS",
+    "device_status", "launch_count", "debug_wait_timeout", "read_bandwidth_probe", "library_path", "load_library", "EXPORTED_SYMBOLS",
     "DEV_ERR_BLOCK_ID", "DEV_ERR_CONTEXT", "DEV_ERR_CONTEXT_HINT", "DEV_ERR_SLOT", "DEV_ERR_TIMEOUT",
+    "DEV_ERR_INTERNAL", "BUILD_DEBUG", "build_flags",
     "BlockManager", "BlockManagerError", "DecodeStepPlan", "PrefillStepPlan",
 ]
 
@@ -40,6 +41,8 @@ DEV_ERR_CONTEXT = 0x2
 DEV_ERR_CONTEXT_HINT = 0x4
 DEV_ERR_SLOT = 0x8
 DEV_ERR_TIMEOUT = 0x10
+DEV_ERR_INTERNAL = 0x20
+BUILD_DEBUG = 0x1
 
 _DTYPES = {torch.float16: 1, torch.bfloat16: 2}
 
@@ -50,7 +53,7 @@ EXPORTED_SYMBOLS = (
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_device_blocks", "pa_bm_num_free_host_blocks",
     "pa_bm_ref_count", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_num_tokens",
     "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step", "pa_bm_build_prefill_step", "pa_bm_step_needs",
-    "pa_bm_swap_out", "pa_bm_swap_in", "pa_prefill",
+    "pa_bm_swap_out", "pa_bm_swap_in", "pa_prefill", "pa_read_bandwidth_probe", "pa_build_flags",
 )
 
 
@@ -59,7 +62,9 @@ class PagedAttentionError(RuntimeError):
 
 
 def library_path() -> str:
-    return _LIB_PATH
+    """The library this process loads: ``PA_B200_LIBRARY`` if set (e.g. the PA_DEBUG build,
+    ``libpa_b200_debug.so``), else the in-tree release build."""
+    return os.environ.get("PA_B200_LIBRARY") or _LIB_PATH
 
 
 def load_library(path: str | None = None) -> ctypes.CDLL:
@@ -68,7 +73,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     with _lock:
         if _lib is not None and path is None:
             return _lib
-        p = path or _LIB_PATH
+        p = path or library_path()
         if not os.path.exists(p):
             raise PagedAttentionError(
                 f"CUDA library {p} is missing; build it with `python -m paged_kv_cache_457_b200.build_lib`")
@@ -101,6 +106,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_prefill.restype = ctypes.c_int
         lib.pa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, f32, vp, i32, i64, i32, i32, i32, i32, i64, i32, i32, i64,
                                    i64, i32, vp]
+        lib.pa_read_bandwidth_probe.restype = ctypes.c_int
+        lib.pa_read_bandwidth_probe.argtypes = [vp, i64, vp, vp]
+        lib.pa_build_flags.restype = ctypes.c_uint32
+        lib.pa_build_flags.argtypes = []
         lib.pa_version.restype = i32
         lib.pa_version.argtypes = []
         from .block_manager import bind as _bind_block_manager
@@ -309,6 +318,23 @@ def device_status(clear: bool = True, device: torch.device | None = None) -> int
     _check(load_library().pa_get_device_status(ctypes.byref(val), 1 if clear else 0, _stream(dev)),
            "pa_get_device_status")
     return int(val.value)
+
+
+def read_bandwidth_probe(buf: torch.Tensor, sink: torch.Tensor) -> None:
+    """Stream every byte of ``buf`` (a contiguous CUDA tensor) through the SMs once, read-only;
+    ``sink`` is a one-element int32 CUDA tensor the kernel folds the data into."""
+    _need_cuda("buf", buf)
+    _need_cuda("sink", sink, buf.device)
+    if not buf.is_contiguous() or sink.dtype != torch.int32 or sink.numel() < 1:
+        raise PagedAttentionError("buf must be contiguous and sink an int32 tensor")
+    nbytes = buf.numel() * buf.element_size() // 16 * 16
+    _check(load_library().pa_read_bandwidth_probe(buf.data_ptr(), nbytes, sink.data_ptr(), _stream(buf.device)),
+           "pa_read_bandwidth_probe")
+
+
+def build_flags() -> int:
+    """BUILD_* bits of the loaded library (BUILD_DEBUG: the PA_DEBUG build)."""
+    return int(load_library().pa_build_flags())
 
 
 def launch_count() -> int:

@@ -1,6 +1,9 @@
 """Builds the in-tree CUDA library ``libpa_b200.so`` for sm_100a with nvcc.
 
-Run ``python -m paged_kv_cache_457_b200.build_lib`` (or ``__graft_entry__.build()``).
+Run ``python -m paged_kv_cache_457_b200.build_lib [--debug]`` (or ``__graft_entry__.build()``, which
+builds both).  ``--debug`` builds ``libpa_b200_debug.so`` with PA_DEBUG: the kernels check every index
+they derive before using it and report a failed check in the device status word
+(PA_DEV_ERR_INTERNAL) instead of touching memory; load it with ``PA_B200_LIBRARY=<path>``.
 """
 from __future__ import annotations
 
@@ -14,8 +17,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpa_b200.so")
+# the same sources with PA_DEBUG: every index the kernels derive is checked on the device before use
+DEBUG_LIB = os.path.join(PKG, "libpa_b200_debug.so")
 SOURCES = [os.path.join(CSRC, "pa_api.cu"), os.path.join(CSRC, "block_manager.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_mma.cuh", "pa_ptx.cuh", "pa_copy.cuh", "pa_prefill.cuh", "pa_tcgen05.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_mma.cuh", "pa_ptx.cuh", "pa_copy.cuh", "pa_prefill.cuh", "pa_tcgen05.cuh", "pa_stream.cuh")] + [
     os.path.join(INCLUDE, h) for h in ("pa_b200.h", "pa_block_manager.h")]
 
 
@@ -26,9 +31,11 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA library cannot be built")
 
 
-def command(out: str = LIB, verbose_ptxas: bool = False) -> list:
+def command(out: str = LIB, verbose_ptxas: bool = False, debug: bool = False) -> list:
     cmd = [nvcc(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
            "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-o", out] + SOURCES
+    if debug:
+        cmd[1:1] = ["-DPA_DEBUG"]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     return cmd
@@ -41,12 +48,13 @@ def up_to_date(out: str = LIB) -> bool:
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if force or verbose_ptxas or not up_to_date():
-        subprocess.run(command(verbose_ptxas=verbose_ptxas), check=True)
-    return LIB
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    out = DEBUG_LIB if debug else LIB
+    if force or verbose_ptxas or not up_to_date(out):
+        subprocess.run(command(out, verbose_ptxas=verbose_ptxas, debug=debug), check=True)
+    return out
 
 
 if __name__ == "__main__":
-    build(force=True, verbose_ptxas="-v" in sys.argv)
-    print(LIB)
+    debug = "--debug" in sys.argv
+    print(build(force=True, verbose_ptxas="-v" in sys.argv, debug=debug))

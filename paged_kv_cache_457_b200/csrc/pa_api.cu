@@ -19,6 +19,7 @@
 #include "pa_kernels.cuh"
 #include "pa_prefill.cuh"
 #include "pa_mma.cuh"
+#include "pa_stream.cuh"
 
 namespace {
 
@@ -768,6 +769,28 @@ int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const in
   if (head_dim == 128) return launch(pa::prefill_tc_kernel<pa::F16, 128>, pa::PrefillSmem<128>::ALLOC);
   return launch(pa::prefill_tc_kernel<pa::F16, 64>, pa::PrefillSmem<64>::ALLOC);
 }
+
+int pa_read_bandwidth_probe(const void *src, int64_t bytes, uint32_t *sink, void *stream) {
+  if (bytes < 0) return PA_ERR_SHAPE;
+  if (bytes == 0) return PA_OK;
+  if (!src || !sink) return PA_ERR_NULL;
+  if (!aligned16(src) || (bytes % 16) || (reinterpret_cast<uintptr_t>(sink) & 3u)) return PA_ERR_ALIGN;
+  int sms = 0;
+  int rc = current_sms(&sms);
+  if (rc != PA_OK) return rc;
+  // four blocks of 512 threads fill an SM's 2048 thread slots
+  const long long n16 = bytes / 16;
+  const long long want = (n16 + pa::STREAM_THREADS - 1) / pa::STREAM_THREADS;
+  const int grid = (int)std::max(1LL, std::min<long long>(want, (long long)sms * 4));
+  pa::stream_read_kernel<<<grid, pa::STREAM_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4 *>(src), n16, reinterpret_cast<unsigned int *>(sink));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return record(e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+uint32_t pa_build_flags(void) { return pa::kDebugChecks ? PA_BUILD_DEBUG : 0u; }
 
 int32_t pa_version(void) { return 100; }
 

@@ -30,6 +30,23 @@ constexpr int TILE = 16;  // tokens per bulk-copied tile
 // Device status word (one per device; see pa_get_device_status).
 __device__ unsigned int g_status = 0;
 
+// Index checks of the debug build (PA_DEBUG): dcheck(ok) flags PA_DEV_ERR_INTERNAL when ok is false and
+// returns ok, so the caller skips the access.  In the release build it is the constant true and the
+// checks compile away.
+#ifdef PA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool dcheck(bool ok) {
+  if constexpr (kDebugChecks) {
+    if (!ok) atomicOr(&g_status, PA_DEV_ERR_INTERNAL);
+    return ok;
+  } else {
+    return true;
+  }
+}
+
 // ---------------------------------------------------------------- element types
 __device__ __forceinline__ float dot8_f16(const uint32_t (&q)[4], const uint4 k, float c);
 __device__ __forceinline__ float dot8_bf16(const uint32_t (&q)[4], const uint4 k, float c);
@@ -111,6 +128,7 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const WriteArgs a) {
     }
     const long long blk = slot / a.block_size;
     const int row = (int)(slot - blk * a.block_size);
+    if (!dcheck(t < a.num_tokens && h < a.num_kv_heads && blk < a.num_blocks && row < a.block_size)) continue;
     const uint16_t *src = (is_v ? a.v + t * a.v_token_stride : a.k + t * a.k_token_stride) + h * a.head_dim + c * 8;
     uint16_t *dst = (is_v ? a.v_cache : a.k_cache) + ((blk * a.num_kv_heads + h) * a.block_size + row) * a.head_dim +
                     c * 8;
@@ -295,6 +313,11 @@ __device__ __forceinline__ TilePos locate_tile(const int *pt, int S, int HC, lon
   TilePos p;
   p.s = lo;
   p.nt = pt[lo + 1] - pt[lo];
+  if (!dcheck(p.nt > 0 && t >= 0 && t < (long long)pt[S] * HC)) {  // a stream position past the tiles
+    p.hc = p.j = 0;
+    p.nt = 1;
+    return p;
+  }
   const long long r = t - (long long)pt[lo] * HC;
   p.hc = (int)(r / p.nt);
   p.j = (int)(r - (long long)p.hc * p.nt);
@@ -348,12 +371,17 @@ struct TileProducer {
         win_nblk = (L + a.block_size - 1) / a.block_size;
       }
       win_base = blk & ~31;
-      ent = (win_base + lane < win_nblk)
+      const bool in_row = dcheck(pos.s < a.num_seqs && win_nblk <= a.table_stride);
+      ent = (in_row && win_base + lane < win_nblk)
                 ? __ldg(a.block_tables + (long long)pos.s * a.table_stride + win_base + lane)
                 : -1;
     }
     const int phys = __shfl_sync(FULL, ent, blk - win_base);
-    return (phys >= 0 && (long long)phys < a.num_blocks) ? phys : -1;
+    if (phys < 0 || (long long)phys >= a.num_blocks) return -1;
+    // the tile's 16 rows lie inside the (block, kv head) slab
+    if (!dcheck(pos.hc / a.n_chunks < a.num_kv_heads && (pos.j * TILE) % a.block_size + TILE <= a.block_size))
+      return -1;
+    return phys;
   }
 
   // Global row (in [num_blocks * num_kv_heads * block_size)) of the tile's first token.
@@ -558,12 +586,14 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
         full = (cp.j == 0 && len == cp.nt);
         slot = (k == 0) ? 0 : 1;
         hq0 = chunk_first_head(a, cp.hc);
-        L = __ldg(a.context_lens + cp.s);
+        const bool q_ok = dcheck(cp.s < S && hq0 + G <= a.num_q_heads);
+        L = q_ok ? __ldg(a.context_lens + cp.s) : 0;
         piece_bad = false;
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4 *>(a.q + (long long)cp.s * a.q_seq_stride +
-                                                                (long long)(hq0 + gg) * D + cl * 8));
+          const uint4 w = q_ok ? __ldg(reinterpret_cast<const uint4 *>(a.q + (long long)cp.s * a.q_seq_stride +
+                                                                       (long long)(hq0 + gg) * D + cl * 8))
+                               : make_uint4(0, 0, 0, 0);
           qw[gg][0] = w.x;
           qw[gg][1] = w.y;
           qw[gg][2] = w.z;
@@ -666,7 +696,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
         }
         if (piece_bad && lane == 0) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
         if (full) {
-          if (lane < LPR) {
+          if (lane < LPR && dcheck(cp.s < S && hq0 + G <= a.num_q_heads)) {
             uint16_t *out_row = a.out + (long long)cp.s * a.out_seq_stride + (long long)hq0 * D + cl * 8;
 #pragma unroll
             for (int gg = 0; gg < G; ++gg) {
@@ -681,8 +711,10 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
           }
         } else {
           const long long prow = (cons_c * 2 + slot) * G;
+          const bool row_ok = dcheck(cons_c < a.max_chunks);
 #pragma unroll
           for (int gg = 0; gg < G; ++gg) {
+            if (!row_ok) break;
             if (lane < LPR && !piece_bad) {
               float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + (prow + gg) * D + cl * 8);
               dst[0] = make_float4(acc[gg][0].x, acc[gg][0].y, acc[gg][1].x, acc[gg][1].y);
@@ -743,8 +775,10 @@ __global__ void __launch_bounds__(256, 1) decode_merge_kernel(const DecodeArgs a
     const ChunkPlan plan = plan_chunks(a, pts);
     const int nt = pt1 - pt0;
     const long long seg0 = (long long)pt0 * HC + (long long)hc * nt;
+    if (!dcheck(nt > 0 && pt0 >= 0 && pt1 <= pts)) return;  // a sequence with a context owns tiles
     const long long c_first = plan.chunk_of(seg0), c_last = plan.chunk_of(seg0 + nt - 1);
     if (c_first == c_last) return;  // one chunk held the whole segment: the split kernel wrote the rows
+    if (!dcheck(c_first >= 0 && c_last < plan.count && c_last < a.max_chunks)) return;
     const int n = (int)(c_last - c_first + 1);
     auto piece_row = [&](int p) -> long long {  // partial row of this warp's first head in piece p
       const long long c = c_first + p;

@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
       if (lane == 0) {
         fence_proxy_async_smem();
         if (phys >= 0) {
-          const int row0 = (int)prod.first_row(a, phys);
+          const int row0 = (int)prod.first_row(a, phys);  // lookup() checked the tile lies in its slab
           unsigned char *dst = ring + st * STAGE_BYTES;
           mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
 #pragma unroll
@@ -196,10 +196,11 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
         full = (cp.j == 0 && len == cp.nt);
         slot = (k == 0) ? 0 : 1;
         hq0 = chunk_first_head(a, cp.hc);
-        L = __ldg(a.context_lens + cp.s);
+        const bool q_ok = dcheck(cp.s < S && hq0 + G <= a.num_q_heads);
+        L = q_ok ? __ldg(a.context_lens + cp.s) : 0;
         piece_bad = false;
         // Q^T as the B operand: b0 = Q[head gid][16ks + 2tig, +1], b1 = the same 8 dims later
-        const bool row_live = gid < G;
+        const bool row_live = gid < G && q_ok;
         const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q + (long long)cp.s * a.q_seq_stride +
                                                                   (long long)(hq0 + (row_live ? gid : 0)) * D);
 #pragma unroll
@@ -314,14 +315,15 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
           for (int mt = 0; mt < KSTEPS; ++mt) {
             const uint32_t t0w = movmatrix_trans(E::narrow2(piece_bad ? 0.f : o[mt][0] * ia, piece_bad ? 0.f : o[mt][1] * ib));
             const uint32_t t1w = movmatrix_trans(E::narrow2(piece_bad ? 0.f : o[mt][2] * ia, piece_bad ? 0.f : o[mt][3] * ib));
-            if (gid < G) {
+            if (gid < G && dcheck(cp.s < S && hq0 + G <= a.num_q_heads)) {
               *reinterpret_cast<uint32_t *>(orow + 16 * mt) = t0w;
               *reinterpret_cast<uint32_t *>(orow + 16 * mt + 8) = t1w;
             }
           }
         } else {
           const long long prow = (cons_c * 2 + slot) * G;
-          if (!piece_bad) {
+          const bool row_ok = dcheck(cons_c < a.max_chunks);
+          if (!piece_bad && row_ok) {
 #pragma unroll
             for (int mt = 0; mt < KSTEPS; ++mt) {
               const int d0 = 16 * mt + gid;
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
               }
             }
           }
-          if (gid == 0) {
+          if (gid == 0 && row_ok) {
             if (ha < G) a.ws_ml[prow + ha] = piece_bad ? make_float2(-INFINITY, -1.f) : make_float2(ma, lta);
             if (hb < G) a.ws_ml[prow + hb] = piece_bad ? make_float2(-INFINITY, -1.f) : make_float2(mb, ltb);
           }

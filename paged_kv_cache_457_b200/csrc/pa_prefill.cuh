@@ -157,7 +157,7 @@ __device__ __forceinline__ int tile_page(const PrefillArgs &a, const PrefillItem
   const int page = j * (PF_BN / bs) + lane;
   int blk = -1;
   *bad = false;
-  if (lane < PF_BN / bs && page * bs < it.kmax) {
+  if (lane < PF_BN / bs && page * bs < it.kmax && dcheck(page < a.table_stride && it.s < a.num_seqs)) {
     blk = a.block_tables[(long long)it.s * a.table_stride + page];
     if (blk < 0 || (long long)blk >= a.num_blocks) {
       *bad = true;
@@ -296,6 +296,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             break;
           }
           it = prefill_item(a, item);
+          if (!dcheck(it.s < a.num_seqs && it.hq < a.num_q_heads)) {
+            it.work = false;
+            it.bad_ctx = false;
+            continue;
+          }
           if (it.past_grid && it.t0 == 0 && it.hq == 0 && lane == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT_HINT);
           if (it.work) break;
           if (!it.bad_ctx && lane == 0) {
@@ -307,6 +312,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           if (it.bad_ctx) {  // zero the item's rows
             if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_CONTEXT);
             for (int r = lane; r < it.rows; r += 32) {
+              if (!dcheck((long long)it.q0 + it.t0 + r < a.num_query_tokens)) break;
               uint4 *dst = reinterpret_cast<uint4 *>(a.out + (long long)(it.q0 + it.t0 + r) * a.out_token_stride +
                                                      (long long)it.hq * D);
 #pragma unroll
@@ -584,7 +590,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         float o[32];
         tc::ld32(t_o + c * 32, o);  // every lane: the load is warp-collective
         tc::wait_ld();
-        if (row < it.rows) {
+        if (row < it.rows && dcheck((long long)it.q0 + it.t0 + row < a.num_query_tokens)) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float f[8];

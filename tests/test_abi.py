@@ -50,6 +50,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.pa_version() == 100
+    assert lib.pa_build_flags() == 0  # the release build; libpa_b200_debug.so reports PA_BUILD_DEBUG
     assert lib.pa_status_string(0) == b"ok"
     for code in range(-9, 0):
         assert lib.pa_status_string(code) != b"unknown status"
