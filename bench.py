@@ -58,7 +58,14 @@ def parse():
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-sample-seconds", type=float, default=10.0,
+                    help="seconds of oracle work per CPU leg (single thread, then all cores)")
+    ap.add_argument("--l2-flush", default="auto", choices=["auto", "on", "off"],
+                    help="auto: write a scratch buffer larger than L2 before every timed step when the step's "
+                         "distinct bytes would fit in L2, else time steps back to back (inputs larger than L2)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time direct library calls instead of replays of a CUDA graph of the step")
+    ap.add_argument("--iters", type=int, default=100, help="per-iteration timings (median, p10, p90)")
     ap.add_argument("--num-seqs", type=int, default=None, help="override (llama2/gqa workloads; profiling)")
     ap.add_argument("--num-blocks", type=int, default=None, help="override (llama2/gqa workloads; profiling)")
     return ap.parse_args()
@@ -123,6 +130,33 @@ def max_over_ranks(values, device=None):
 def job_rate_gbs(bytes_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
     """Whole-job throughput: every rank moves bytes_per_rank_step per step; time = slowest rank."""
     return world * bytes_per_rank_step * steps / (max_ms / 1e3) / 1e9
+
+
+def summarize_ms(times_ms):
+    """Median, p10, p90 and mean (microseconds) of per-iteration times given in milliseconds."""
+    a = np.asarray(times_ms, dtype=np.float64) * 1e3
+    if a.size == 0:
+        return None
+    return {"median_us": round(float(np.median(a)), 3), "p10_us": round(float(np.percentile(a, 10)), 3),
+            "p90_us": round(float(np.percentile(a, 90)), 3), "mean_us": round(float(a.mean()), 3), "n": int(a.size)}
+
+
+def flush_needed(mode: str, distinct_bytes: int, l2_bytes: int) -> bool:
+    """Whether timed steps must be separated by an L2 flush: always ("on"), never ("off"), or when
+    the bytes one step reads (each distinct byte once) are not several times the L2 ("auto")."""
+    if mode == "on":
+        return True
+    if mode == "off":
+        return False
+    return distinct_bytes < 4 * l2_bytes
+
+
+def l2_note(flush: bool, distinct_bytes: int, l2_bytes: int, flush_bytes: int) -> str:
+    size = f"{distinct_bytes / 1e6:.1f} MB of distinct inputs per step against a {l2_bytes / 1e6:.0f} MB L2"
+    if flush:
+        return (f"flushed: a {flush_bytes / 2**20:.0f} MiB scratch write and read-back before every timed step "
+                f"({size})")
+    return f"no flush: {size}, steps back to back"
 
 
 def measured_peak():
@@ -217,6 +251,40 @@ def cpu_oracle_rate(wl, st, seconds: float):
     return done_bytes / elapsed / 1e9, n, elapsed
 
 
+def cpu_oracle_rate_parallel(wl, st, seconds: float):
+    """Times the OpenMP build of the fp64 C oracle on all host cores: batches of one sequence per
+    thread, rotating through the step, until about ``seconds`` have passed; returns
+    (GB/s of KV it processed, threads, description)."""
+    import oracle
+    kc, vc = oracle.write_kv(st.k_new, st.v_new, wl.k_cache, wl.v_cache, st.slot_mapping, wl.block_size)
+    threads = oracle.parallel_threads()
+    per_seq = wl.num_kv_heads * wl.head_dim * 2 * 2
+    batch = max(1, min(threads, st.num_seqs))
+    done_bytes, elapsed, calls, seqs = 0, 0.0, 0, 0
+    while elapsed < seconds:
+        idx = (np.arange(batch) + calls * batch) % st.num_seqs
+        t = time.perf_counter()
+        oracle.decode(st.q[idx], kc, vc, st.block_tables[idx], st.context_lens[idx], wl.scale, wl.dtype,
+                      parallel=True)
+        elapsed += time.perf_counter() - t
+        done_bytes += int(st.context_lens[idx].sum()) * per_seq
+        calls += 1
+        seqs += batch
+    return done_bytes / elapsed / 1e9, threads, (
+        f"{seqs} sequence passes ({calls} calls of {batch} sequences, rotating through the {st.num_seqs} of one "
+        f"step), {elapsed:.1f} s, {threads} OpenMP threads over (sequence, query head)")
+
+
+def cpu_baseline(wl, st, seconds: float):
+    """The oracle timed on the host: all cores (the reported value) and one thread beside it."""
+    rate1, nseq, secs = cpu_oracle_rate(wl, st, seconds)
+    rate_n, threads, sample_n = cpu_oracle_rate_parallel(wl, st, seconds)
+    return {"value": round(rate_n, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample_n,
+            "host_cores_in_affinity": len(os.sched_getaffinity(0)),
+            "single_thread": {"value": round(rate1, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"first {nseq} of {st.num_seqs} sequences of one step, {secs:.1f} s"}}
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -226,26 +294,30 @@ def run_reference(args):
     import oracle
     kc, vc = oracle.write_kv(st.k_new, st.v_new, wl.k_cache, wl.v_cache, st.slot_mapping, wl.block_size)
     per_seq = wl.num_kv_heads * wl.head_dim * 2 * 2
-    # one step = the oracle on a 2-sequence sample of the batch (rotating), bounded work per step
-    sample = 2
+    threads = oracle.parallel_threads()
+    # one step = the oracle on all host cores over a sample of one sequence per thread (rotating through
+    # the batch), so the work per step stays bounded whatever the workload
+    sample = max(1, min(threads, st.num_seqs))
     times, nbytes = [], []
     for i in range(args.warmup + args.steps):
         idx = (np.arange(sample) + i * sample) % st.num_seqs
         t = time.perf_counter()
-        oracle.decode(st.q[idx], kc, vc, st.block_tables[idx], st.context_lens[idx], wl.scale, wl.dtype)
+        oracle.decode(st.q[idx], kc, vc, st.block_tables[idx], st.context_lens[idx], wl.scale, wl.dtype,
+                      parallel=True)
         dt = time.perf_counter() - t
         if i >= args.warmup:
             times.append(dt)
             nbytes.append(int(st.context_lens[idx].sum()) * per_seq)
     total_t = sum(times)
     value = sum(nbytes) / total_t / 1e9
+    desc = f"{sample} of {st.num_seqs} sequences per step, rotating; {threads} OpenMP threads"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_t / len(times), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "description": wl.description, "sample": f"{sample} sequences per step"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{sample} of {st.num_seqs} sequences per step, rotating"},
+        "config": {"workload": wl.name, "description": wl.description, "sample": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": desc, "host_cores_in_affinity": len(os.sched_getaffinity(0))},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -680,40 +752,129 @@ def main():
                   partition_tokens=part, workspace=ws)
 
     kv_b, alg_b = step_bytes(wl, st)
+    uniq_kv = W.unique_kv_bytes(st, wl.num_kv_heads, wl.head_dim, wl.block_size)
+    alg_unique = alg_b - kv_b + uniq_kv  # shared prefix blocks counted once: what must come from HBM
+    l2_bytes = int(torch.cuda.get_device_properties(device).L2_cache_size)
+    flush = flush_needed(args.l2_flush, alg_unique, l2_bytes)
+    flush_bytes = max(512 * 2**20, 4 * l2_bytes)
+    flush_buf = torch.empty(flush_bytes, dtype=torch.uint8, device=device) if flush else None
     torch.cuda.synchronize()
     assert pa.device_status() == 0, "device status after setup"
 
+    # The step as a CUDA graph (default): one replay re-runs the library's kernels with the captured
+    # arguments, so the host's per-call cost (argument checks, ctypes) is paid once, at capture.
+    reference_out = None
+    launches_per_step = 3
+    if not args.no_graph:
+        step()
+        torch.cuda.synchronize()
+        reference_out = out.clone()
+        graph = torch.cuda.CUDAGraph()
+        n0 = pa.launch_count()
+        with torch.cuda.graph(graph):
+            step()
+        launches_per_step = pa.launch_count() - n0
+        run_step = graph.replay
+    else:
+        run_step = step
+
+    def prime():
+        # a GPU-side wait ahead of the timed region, so the host enqueues the timed steps while the GPU is
+        # busy: the clock then measures the GPU's work, not the host's launch rate
+        torch.cuda._sleep(50_000_000)
+
+    flush_sink = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def flush_l2(i):
+        # write a buffer several times the L2, then read it back: the read pass evicts the written lines
+        # (their write-back to HBM happens here, not inside the timed step), so L2 holds only clean
+        # lines of the scratch buffer when the step starts
+        flush_buf.fill_(i & 0x7f)
+        pa.read_bandwidth_probe(flush_buf, flush_sink)
+
+    def timed_per_iteration(fn, n, cold):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        prime()
+        for i in range(n):
+            if cold:
+                flush_l2(i)
+            evs[i][0].record()
+            fn()
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
     sampler = ClockSampler(device).start()
     for _ in range(args.warmup):
-        step()
+        run_step()
     torch.cuda.synchronize()
+    if reference_out is not None:
+        assert torch.equal(out, reference_out), "graph replay differs from the direct call"
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = pa.launch_count()
     wall0 = time.perf_counter()
-    t_start.record()
-    for _ in range(args.steps):
-        step()
-    t_end.record()
-    torch.cuda.synchronize()
+    if flush:
+        step_times = timed_per_iteration(run_step, args.steps, cold=True)
+        elapsed_ms = float(sum(step_times))
+    else:
+        prime()
+        t_start.record()
+        for _ in range(args.steps):
+            run_step()
+        t_end.record()
+        torch.cuda.synchronize()
+        elapsed_ms = t_start.elapsed_time(t_end)
+        step_times = None
     wall1 = time.perf_counter()
     launches = pa.launch_count() - launches0
+    if flush:
+        launches -= args.steps  # the flush's read-back pass between steps is not part of a step
+    if not args.no_graph:
+        launches = launches_per_step * args.steps  # replays do not pass through the host-side counter
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    # the dominant kernels alone: K back-to-back pa_decode calls (split + merge), same inputs
+
+    # pa_decode alone (split + merge kernels), the roofline's kernel: back to back, then per iteration with
+    # and without an L2 flush before each call
+    if not args.no_graph:
+        dgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(dgraph):
+            decode_only()
+        run_decode = dgraph.replay
+    else:
+        run_decode = decode_only
+    for _ in range(3):
+        run_decode()
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    prime()
     d0.record()
     for _ in range(args.steps):
-        decode_only()
+        run_decode()
     d1.record()
     torch.cuda.synchronize()
-    dec_ms = d0.elapsed_time(d1) / args.steps
+    dec_b2b_ms = d0.elapsed_time(d1) / args.steps
+    if flush_buf is None:
+        flush_buf = torch.empty(flush_bytes, dtype=torch.uint8, device=device)
+    cold = timed_per_iteration(run_decode, args.iters, cold=True)
+    warm = timed_per_iteration(run_decode, args.iters, cold=False)
+    dec_ms = float(np.mean(cold)) if flush else dec_b2b_ms
+    del flush_buf
     status = pa.device_status()
+
+    # read-only streaming rate of this GPU, measured now by the library's own probe kernel
+    probe_bytes = max(2 * 2**30, 8 * l2_bytes)
+    probe_buf = torch.empty(probe_bytes, dtype=torch.uint8, device=device)
+    sink = torch.zeros(1, dtype=torch.int32, device=device)
+    for _ in range(3):
+        pa.read_bandwidth_probe(probe_buf, sink)
+    probe_ms = timed_per_iteration(lambda: pa.read_bandwidth_probe(probe_buf, sink), 20, cold=False)
+    read_peak = probe_bytes / (min(probe_ms) / 1e3) / 1e9
+    del probe_buf
 
     # ---- end to end through the public API: pinned host inputs -> device -> step -> host output
     e2e = None
@@ -786,37 +947,66 @@ def main():
                "how": "each step's inputs copied from pinned host memory and its output read back, on two copy "
                       "streams, double-buffered so that they overlap the previous step's kernels"}
 
-    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], device)
+    elapsed_ms, dec_ms, read_peak_neg = max_over_ranks([elapsed_ms, dec_ms, -read_peak], device)
+    read_peak = -read_peak_neg  # the slowest rank's probe
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, nseq, secs = cpu_oracle_rate(wl, st, args.cpu_sample_seconds)
-        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"first {nseq} of {st.num_seqs} sequences of one step, {secs:.1f} s, single thread"}
+        cpu = cpu_baseline(wl, st, args.cpu_sample_seconds)
 
     if rank == 0:
         ms_step = elapsed_ms / args.steps
         value = job_rate_gbs(kv_b, world, args.steps, elapsed_ms)
+        value_distinct = job_rate_gbs(uniq_kv, world, args.steps, elapsed_ms)
         peak, peak_kind = measured_peak()
-        achieved = alg_b / (dec_ms / 1e3) / 1e9
+        achieved = alg_unique / (dec_ms / 1e3) / 1e9
         traffic, traffic_note = recorded_traffic(wl.name)
+        shared = uniq_kv != kv_b
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "storage_dtype": wl.dtype, "data": "synthetic",
             "seq_steps_per_s": round(world * st.num_seqs / (ms_step / 1e3), 1),
-            "frac_of_hbm_peak": round(value / world / peak, 4),
-            "frac_of_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
+            "distinct_kv_gbs": round(value_distinct, 2),
+            "frac_of_hbm_peak": round(value_distinct / world / peak, 4),
+            "frac_of_read_only_peak": round(value_distinct / world / read_peak, 4),
+            "frac_of_8tbs": round(value_distinct / world / NOMINAL_HBM_GBS, 4),
             "config": {"workload": wl.name, "description": wl.description, "num_seqs": st.num_seqs,
                        "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                        "block_size": wl.block_size, "max_context_len": mcl,
                        "split": f"chunks of {part} tokens" if part else "balanced (one chunk of tiles per warp)",
-                       "kv_bytes_per_step": kv_b, "parallelism": f"dp{world} (independent batches per GPU)",
-                       "l2": f"no flush: {kv_b / 1e9:.2f} GB of K/V per step, larger than the 126 MB L2"},
+                       "kv_bytes_per_step": kv_b, "distinct_kv_bytes_per_step": uniq_kv,
+                       "parallelism": f"dp{world} (independent batches per GPU)",
+                       "timing": ("per-step CUDA events, L2 flushed before each step" if flush else
+                                  "one CUDA event pair around all steps, back to back")
+                       + ("; each step a replay of a CUDA graph of pa_write_kv + pa_decode" if not args.no_graph
+                          else "; direct library calls"),
+                       "l2": l2_note(flush, alg_unique, l2_bytes, flush_bytes)},
+            "step_timing": summarize_ms(step_times) if step_times else None,
             "roofline": {"bound": "hbm", "kernel": "pa_decode (split + merge kernels)",
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_note": traffic_note,
-                         "algorithmic_bytes": alg_b, "ms_per_launch": round(dec_ms, 5)},
+                         "algorithmic_bytes": alg_unique,
+                         "algorithmic_bytes_note": ("K/V of the distinct physical rows read (a prefix block named by "
+                                                    "several tables counted once) + q + out + table entries + lengths"
+                                                    if shared else "K/V of the live tokens + q + out + table entries "
+                                                    "+ lengths"),
+                         "ms_per_launch": round(dec_ms, 5),
+                         "launch_timing": "mean of per-call times, L2 flushed before each call" if flush else
+                                          "back-to-back calls, mean",
+                         "peaks": {
+                             "measured_copy": {"gbs": peak, "frac": round(achieved / peak, 4),
+                                               "source": "MEASURED_PEAKS.json hbm_gbs (read+write copy)"},
+                             "read_only_probe": {"gbs": round(read_peak, 1), "frac": round(achieved / read_peak, 4),
+                                                 "source": "pa_read_bandwidth_probe over "
+                                                           f"{probe_bytes / 2**30:.1f} GiB, best of 20, this run"},
+                             "nominal_8tbs": {"gbs": NOMINAL_HBM_GBS, "frac": round(achieved / NOMINAL_HBM_GBS, 4)}},
+                         "logical_bytes": alg_b if shared else None,
+                         "logical_rate_note": (f"{alg_b / (dec_ms / 1e3) / 1e9:.1f} GB/s counting every table's "
+                                               "reads of the shared prefix; not a fraction of any peak (repeat reads "
+                                               "of a block come from L2)") if shared else None},
+            "decode_timing": {"back_to_back_us": round(dec_b2b_ms * 1e3, 3), "cold_l2": summarize_ms(cold),
+                              "warm_l2": summarize_ms(warm)},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": sampler.summary(wall0, wall1), "device_status": status,
         }

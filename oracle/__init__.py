@@ -35,8 +35,10 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "pa_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libpa_oracle.so")
+_OMP_LIB_PATH = os.path.join(_HERE, "libpa_oracle_omp.so")
 _lock = threading.Lock()
 _lib = None
+_omp_lib = None
 
 DTYPE_CODES = {"fp16": 1, "bf16": 2}
 
@@ -54,6 +56,24 @@ def build(src: str = _SRC, out: str = _LIB_PATH) -> str:
     cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math", "-o", out, src, "-lm"]
     subprocess.run(cmd, check=True)
     return out
+
+
+def build_parallel(src: str = _SRC, out: str = _OMP_LIB_PATH) -> str:
+    """Compile the same source with OpenMP: only ``oracle_decode_parallel`` changes, from one
+    thread to all the host's cores; its arithmetic per (sequence, query head) is unchanged."""
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math", "-fopenmp", "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _load_parallel() -> ctypes.CDLL:
+    global _omp_lib
+    with _lock:
+        if _omp_lib is None:
+            if (not os.path.exists(_OMP_LIB_PATH)) or os.path.getmtime(_OMP_LIB_PATH) < os.path.getmtime(_SRC):
+                build_parallel()
+            _omp_lib = _bind(ctypes.CDLL(_OMP_LIB_PATH))
+        return _omp_lib
 
 
 def _load(path: str | None = None) -> ctypes.CDLL:
@@ -76,6 +96,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_decode.restype = ctypes.c_int
     lib.oracle_decode.argtypes = [p, p, p, p, i64, p, i64, i64, i64, i64, i64, i64, ctypes.c_int,
                                   ctypes.c_double, p]
+    lib.oracle_decode_parallel.restype = ctypes.c_int
+    lib.oracle_decode_parallel.argtypes = lib.oracle_decode.argtypes
+    lib.oracle_parallel_threads.restype = ctypes.c_int
+    lib.oracle_parallel_threads.argtypes = []
     lib.oracle_prefill.restype = ctypes.c_int
     lib.oracle_prefill.argtypes = [p, p, p, p, i64, p, p, i64, i64, i64, i64, i64, i64, ctypes.c_int,
                                    ctypes.c_double, p]
@@ -133,9 +157,13 @@ def write_kv(k, v, k_cache, v_cache, slot_mapping, block_size: int, lib_path: st
 
 
 def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype: str,
-           lib_path: str | None = None) -> np.ndarray:
-    """Exact (fp64) paged decode attention; returns float64 [S, Hq, d]."""
-    lib = _load(lib_path)
+           lib_path: str | None = None, parallel: bool = False) -> np.ndarray:
+    """Exact (fp64) paged decode attention; returns float64 [S, Hq, d].
+
+    ``parallel=True`` runs the OpenMP build over all host cores (same arithmetic, same bits);
+    it exists to time the oracle on every core."""
+    lib = _load_parallel() if parallel else _load(lib_path)
+    fn = lib.oracle_decode_parallel if parallel else lib.oracle_decode
     q = _u16(q, "q")
     kc = _u16(k_cache, "k_cache")
     vc = _u16(v_cache, "v_cache")
@@ -150,11 +178,16 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype:
     out = np.zeros((S, hq, d), dtype=np.float64)
     if S == 0:
         return out
-    rc = lib.oracle_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), bt.shape[1], _ptr(cl), S, hq, hkv, d, bs,
-                           nb, DTYPE_CODES[dtype], float(scale), _ptr(out))
+    rc = fn(_ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), bt.shape[1], _ptr(cl), S, hq, hkv, d, bs,
+            nb, DTYPE_CODES[dtype], float(scale), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle_decode: {ERRORS.get(rc, rc)}")
     return out
+
+
+def parallel_threads() -> int:
+    """Threads the OpenMP build of the decode uses on this host."""
+    return int(_load_parallel().oracle_parallel_threads())
 
 
 def copy_blocks(src_k, src_v, dst_k, dst_v, mapping, lib_path: str | None = None):

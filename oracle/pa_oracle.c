@@ -37,6 +37,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORACLE_OK 0
 #define ORACLE_ERR_ARG -1
@@ -199,6 +202,73 @@ int oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_
 done:
     free(K); free(V); free(z);
     return rc;
+}
+
+/*
+ * The same decode, with the (sequence, query head) pairs shared among the
+ * host's cores by OpenMP when this file is compiled with -fopenmp (without
+ * it the pragmas are ignored and the loop runs on one thread).  Each pair
+ * runs exactly the steps of oracle_decode -- gather through the table, then
+ * attend -- on buffers private to its thread, so the results are identical
+ * to oracle_decode's, bit for bit, whatever the thread count.  Used only to
+ * time the oracle on every core; the checks of the GPU path use
+ * oracle_decode.
+ */
+int oracle_decode_parallel(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                           const int32_t *block_tables, int64_t table_stride, const int32_t *context_lens,
+                           int64_t num_seqs, int64_t num_q_heads, int64_t num_kv_heads, int64_t head_dim,
+                           int64_t block_size, int64_t num_blocks, int dtype, double scale, double *out) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_q_heads % num_kv_heads != 0 || (dtype != 1 && dtype != 2))
+        return ORACLE_ERR_ARG;
+    int64_t max_len = 0;
+    for (int64_t s = 0; s < num_seqs; ++s) {
+        int64_t L = context_lens[s];
+        if (L < 0 || L > table_stride * block_size) return ORACLE_ERR_CONTEXT;
+        for (int64_t j = 0; j < L; j += block_size) {
+            int32_t p = block_tables[s * table_stride + j / block_size];
+            if (p < 0 || p >= num_blocks) return ORACLE_ERR_BLOCK_ID;
+        }
+        if (L > max_len) max_len = L;
+    }
+    int64_t group = num_q_heads / num_kv_heads;
+    int64_t pairs = num_seqs * num_q_heads;
+    int rc = ORACLE_OK;
+#pragma omp parallel
+    {
+        size_t cap = (size_t)(max_len > 0 ? max_len : 1);
+        double *K = (double *)malloc(cap * (size_t)head_dim * sizeof(double));
+        double *V = (double *)malloc(cap * (size_t)head_dim * sizeof(double));
+        double *z = (double *)malloc(cap * sizeof(double));
+        int ok = K && V && z;
+        if (!ok) {
+#pragma omp atomic write
+            rc = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t u = 0; u < pairs; ++u) {
+            int64_t s = u / num_q_heads, hq = u % num_q_heads;
+            int64_t L = context_lens[s];
+            double *o = out + (s * num_q_heads + hq) * head_dim;
+            for (int64_t i = 0; i < head_dim; ++i) o[i] = 0.0;
+            if (L == 0 || !ok) continue;
+            const uint16_t *qrow = q + u * head_dim;  /* u = s * num_q_heads + hq */
+            gather_rows(k_cache, v_cache, block_tables + s * table_stride, L, hq / group, num_kv_heads, head_dim,
+                        block_size, dtype, K, V);
+            attend(qrow, K, V, L, head_dim, dtype, scale, z, o);
+        }
+        free(K); free(V); free(z);
+    }
+    return rc;
+}
+
+/* Threads oracle_decode_parallel uses (1 when compiled without OpenMP). */
+int oracle_parallel_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /*

@@ -82,7 +82,7 @@ def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "GB/s"
     assert line["value"] > 0 and line["higher_is_better"] is True and line["steps"] == 2
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
 
 
@@ -95,3 +95,27 @@ def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
                                       "--steps", "2", "--warmup", "1"])
     assert bench.main() == 0
     assert capsys.readouterr().out.strip() == ""
+
+
+def test_flush_rule_and_note():
+    l2 = 126 * 10**6
+    assert bench.flush_needed("auto", 67 * 10**6, l2)        # a shared-prefix step fits in L2: flush
+    assert not bench.flush_needed("auto", 1_200 * 10**6, l2)  # the Llama-2 batch streams 10x the L2
+    assert bench.flush_needed("on", 10**10, l2) and not bench.flush_needed("off", 1, l2)
+    assert "flushed" in bench.l2_note(True, 10**6, l2, 512 * 2**20)
+    assert "no flush" in bench.l2_note(False, 10**9, l2, 512 * 2**20)
+
+
+def test_summary_of_per_iteration_times():
+    s = bench.summarize_ms([0.010] * 8 + [0.020, 0.030])
+    assert s["median_us"] == pytest.approx(10.0) and s["n"] == 10
+    assert s["p10_us"] <= s["median_us"] <= s["p90_us"]
+    assert s["mean_us"] == pytest.approx(13.0)
+
+
+def test_shared_prefix_distinct_bytes_below_logical():
+    wl = W.shared_prefix()
+    st = wl.steps[1]
+    kv, _ = bench.step_bytes(wl, st)
+    uniq = W.unique_kv_bytes(st, wl.num_kv_heads, wl.head_dim, wl.block_size)
+    assert uniq < kv / 3  # 8 tables name each prefix block
