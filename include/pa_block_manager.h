@@ -121,7 +121,11 @@ int pa_bm_append_slot(pa_block_manager *bm, int64_t seq_id, int64_t *slot, int64
  * The pairs never overlap (each destination is a fresh page), so one
  * pa_copy_blocks call applies them.  The whole step fails without change if
  * the pool runs out, a table is longer than table_stride, or the copy array
- * is too small (num_seqs pairs always suffice). */
+ * is too small (num_seqs pairs always suffice).  The one exception:
+ * *num_copies is written as soon as the step is planned, so on
+ * PA_BM_ERR_NO_SPACE, or PA_BM_ERR_CAPACITY from a too-small copy array, it
+ * holds the number of pairs the step needs (to size copy_pairs with); on
+ * earlier failures it is left as it was. */
 int pa_bm_build_decode_step(pa_block_manager *bm, const int64_t *seq_ids, int64_t num_seqs, int64_t table_stride,
                             int32_t *block_tables, int32_t *context_lens, int64_t *slot_mapping,
                             int64_t *copy_pairs, int64_t copy_capacity, int64_t *num_copies);
@@ -144,7 +148,9 @@ int pa_bm_build_decode_step(pa_block_manager *bm, const int64_t *seq_ids, int64_
  * A sequence with no new tokens gets its table and length only.  The whole
  * step fails without change if the pool runs out, a table is longer than
  * table_stride, a length or the token total passes int32, or an output array
- * is too small. */
+ * is too small; as for pa_bm_build_decode_step, *num_copies alone is written
+ * once the step is planned (on PA_BM_ERR_NO_SPACE or a too-small slot or copy
+ * array it holds the pairs the step needs). */
 int pa_bm_build_prefill_step(pa_block_manager *bm, const int64_t *seq_ids, const int64_t *new_tokens,
                              int64_t num_seqs, int64_t table_stride, int32_t *block_tables, int32_t *query_start,
                              int32_t *context_lens, int64_t *slot_mapping, int64_t slot_capacity,

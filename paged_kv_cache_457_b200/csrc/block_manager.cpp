@@ -88,19 +88,18 @@ struct pa_block_manager {
 
   // Plan of a step in which sequence i brings new_tokens[i] >= 0 tokens: the fresh device pages and the
   // copy-on-write pairs its appends will take (simulating the references that earlier copies of the same
-  // step drop from shared last pages), the token total, and the sequences in order.  Tables longer than
-  // table_stride fail with PA_BM_ERR_CAPACITY.  Changes nothing.
+  // step drop from shared last pages) and the token total.  Tables longer than table_stride fail with
+  // PA_BM_ERR_CAPACITY.  A const member: planning cannot change the pool.
   int plan_step(const int64_t *ids, const int64_t *new_tokens, int64_t n, int64_t table_stride, int64_t *pages,
-                int64_t *copies, int64_t *total, std::vector<Seq *> *list) {
-    list->reserve(static_cast<size_t>(n));
+                int64_t *copies, int64_t *total) const {
     std::unordered_set<int64_t> seen;
     std::unordered_map<int32_t, int32_t> dropped;
     const int64_t int32_max = std::numeric_limits<int32_t>::max();
     *pages = *copies = *total = 0;
     for (int64_t i = 0; i < n; ++i) {
-      auto it = seqs.find(ids[i]);
+      const auto it = seqs.find(ids[i]);
       if (it == seqs.end()) return PA_BM_ERR_UNKNOWN;
-      auto &s = it->second;
+      const Seq &s = it->second;
       if (s.host) return PA_BM_ERR_STATE;
       if (!seen.insert(ids[i]).second) return PA_BM_ERR_ARG;
       const int64_t add = new_tokens[i];
@@ -116,7 +115,6 @@ struct pa_block_manager {
         *pages += pages_for(s.tokens + add) - pages_for(s.tokens);
       }
       if (pages_for(s.tokens + add) > table_stride) return PA_BM_ERR_CAPACITY;
-      list->push_back(&s);
     }
     return PA_BM_OK;
   }
@@ -392,14 +390,17 @@ int pa_bm_build_prefill_step(pa_block_manager *bm, const int64_t *seq_ids, const
       return PA_BM_ERR_ARG;
     if (num_seqs > 0 && (!seq_ids || !new_tokens || !context_lens || (table_stride > 0 && !block_tables)))
       return PA_BM_ERR_ARG;
-    std::vector<pa_block_manager::Seq *> list;
     int64_t pages = 0, copies = 0, total = 0;
-    const int rc = bm->plan_step(seq_ids, new_tokens, num_seqs, table_stride, &pages, &copies, &total, &list);
+    const int rc = bm->plan_step(seq_ids, new_tokens, num_seqs, table_stride, &pages, &copies, &total);
     if (rc != PA_BM_OK) return rc;
     *num_copies = copies;
     if (pages > bm->dev.num_free()) return PA_BM_ERR_NO_SPACE;
     if (total > slot_capacity || (total > 0 && !slot_mapping)) return PA_BM_ERR_CAPACITY;
     if (copies > copy_capacity || (copies > 0 && !copy_pairs)) return PA_BM_ERR_CAPACITY;
+    // the planned sequences (all present: planning checked every id)
+    std::vector<pa_block_manager::Seq *> list;
+    list.reserve(static_cast<size_t>(num_seqs));
+    for (int64_t i = 0; i < num_seqs; ++i) list.push_back(&bm->seqs.find(seq_ids[i])->second);
     for (int64_t i = 0; i < num_seqs; ++i) {
       auto *s = list[static_cast<size_t>(i)];
       s->table.reserve(static_cast<size_t>(bm->pages_for(s->tokens + new_tokens[i])));
@@ -435,12 +436,8 @@ int pa_bm_step_needs(const pa_block_manager *bm, const int64_t *seq_ids, const i
   try {
     std::lock_guard<std::mutex> g(bm->mu);
     if (num_seqs < 0 || !pages || !copies || (num_seqs > 0 && (!seq_ids || !new_tokens))) return PA_BM_ERR_ARG;
-    std::vector<pa_block_manager::Seq *> list;
     int64_t total = 0;
-    // plan_step reads the state only; the cast lets it hand back the sequences it planned for
-    return const_cast<pa_block_manager *>(bm)->plan_step(seq_ids, new_tokens, num_seqs,
-                                                          std::numeric_limits<int64_t>::max(), pages, copies,
-                                                          &total, &list);
+    return bm->plan_step(seq_ids, new_tokens, num_seqs, std::numeric_limits<int64_t>::max(), pages, copies, &total);
   } catch (const std::bad_alloc &) {
     return PA_BM_ERR_HOST_MEMORY;
   }

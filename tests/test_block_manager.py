@@ -339,10 +339,10 @@ def test_concurrent_calls_keep_the_pool_consistent():
     def worker(base):
         rng = np.random.default_rng(base)
         mine = []
-        try:
-            for i in range(300):
-                sid = base * 100000 + i
-                r = rng.random()
+        for i in range(300):
+            sid = base * 100000 + i
+            r = rng.random()
+            try:
                 if r < 0.4 or not mine:
                     bm.add_sequence(sid, int(rng.integers(0, 80)))
                     mine.append(sid)
@@ -354,15 +354,22 @@ def test_concurrent_calls_keep_the_pool_consistent():
                 elif r < 0.85:  # a chunk for a few of this thread's sequences
                     pick = [int(x) for x in rng.choice(mine, size=min(3, len(mine)), replace=False)]
                     chunk = [int(x) for x in rng.integers(0, 40, size=len(pick))]
-                    bm.step_needs(pick, chunk)
-                    bm.build_prefill_step(pick, chunk, 256)
+                    # the copies a step needs depend only on pages this thread's own sequences share
+                    # (each thread forks only its own), so the prediction holds under contention
+                    _, copies = bm.step_needs(pick, chunk)
+                    plan = bm.build_prefill_step(pick, chunk, 256)
+                    if len(plan.copy_pairs) != copies:
+                        errors.append(AssertionError(f"step_needs said {copies} copies, the step made "
+                                                     f"{len(plan.copy_pairs)}"))
                 else:
                     victim = int(rng.choice(mine))
                     bm.free_sequence(victim)
                     mine.remove(victim)
-        except BlockManagerError as e:
-            if e.code != -21:  # running out of pages is allowed under contention; anything else is not
-                errors.append(e)
+            except BlockManagerError as e:
+                # running out of pages is allowed under contention (that operation changed nothing, and
+                # the thread goes on); anything else is not
+                if e.code != -21:
+                    errors.append(e)
         return mine
 
     results = {}
