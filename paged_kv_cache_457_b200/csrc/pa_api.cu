@@ -95,7 +95,11 @@ int device_view(const void *p, const void **out) {
 // Query heads handled together by one head chunk (the K/V tiles are read once
 // for all of them).  Groups of 1 or 2 run on the CUDA-core kernel; larger
 // groups run on the tensor-core kernel, whose chunks take up to 8 query heads
-// (the largest divisor of the group size not above 8).
+// (the largest divisor of the group size not above 8).  Measured on B200 with
+// the CUDA-core kernel extended to 3 and 4 heads per chunk: 287 us against
+// 165 us for the 32 query / 8 kv head batch (256 sequences) and 112 us against
+// 45 us for the shared-prefix step (the extra accumulators spill at head_dim
+// 128, and the fp32 FMA work per K/V byte doubles).
 bool uses_mma(int group) { return group >= 3; }
 int heads_per_unit(int group) {
   if (!uses_mma(group)) return group;
@@ -183,6 +187,23 @@ uint32_t split_smem(int head_dim, int group, int num_seqs) {
                          : pa::SplitSmem<kWarps, kStages, 2 * pa::TILE * 64 * 2>::bytes(num_seqs);
 }
 
+// The per-segment kernel (small batches, CUDA-core path): one block of kWarps warps per segment.
+template <class E, int D>
+const void *segment_kernel(int G) {
+  if (G == 2) return reinterpret_cast<const void *>(pa::decode_segment_kernel<E, D, 2, kWarps, kStages>);
+  return reinterpret_cast<const void *>(pa::decode_segment_kernel<E, D, 1, kWarps, kStages>);
+}
+const void *segment_kernel_for(int dtype, int head_dim, int G) {
+  if (dtype == PA_BFLOAT16) return head_dim == 128 ? segment_kernel<pa::BF16, 128>(G) : segment_kernel<pa::BF16, 64>(G);
+  return head_dim == 128 ? segment_kernel<pa::F16, 128>(G) : segment_kernel<pa::F16, 64>(G);
+}
+uint32_t segment_smem(int head_dim) {
+  return head_dim == 128 ? pa::SplitSmem<kWarps, kStages, 2 * pa::TILE * 128 * 2>::bytes(0)
+                         : pa::SplitSmem<kWarps, kStages, 2 * pa::TILE * 64 * 2>::bytes(0);
+}
+// A segment of at most this many 16-token tiles (kWarps warps x 8) may take the per-segment kernel.
+constexpr int kSegmentMaxTiles = kWarps * 8;
+
 // Resident blocks per SM of `kernel` with `smem` bytes of dynamic shared memory (cached).
 struct OccEntry {
   int dev;
@@ -237,6 +258,7 @@ int check_decode_shape(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_hea
 // size does not depend on the storage type: it is sized for the larger of the
 // two instantiations' grids, and the launch never uses more warps than that.
 struct LaunchPlan {
+  bool segment_mode;  // the per-segment kernel, no workspace, no merge kernel
   uint32_t smem;
   int grid;          // blocks of the split kernel (for `dtype`; 0 if not asked)
   long long max_chunks;
@@ -252,6 +274,26 @@ int plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, i
   if (rc != PA_OK) return rc;
   const int group = num_q_heads / num_kv_heads;
   const int G = heads_per_unit(group);
+  // Small batches on the CUDA-core path: every segment (sequence, head chunk) fits one wave of per-segment
+  // blocks and has at most kSegmentMaxTiles tiles.  The choice depends on the sizes only, not on the
+  // storage type, so the workspace size query agrees with the call.
+  lp->segment_mode = false;
+  if (!uses_mma(group) && partition_tokens == 0 && num_seqs > 0 &&
+      ((long long)max_context_len + pa::TILE - 1) / pa::TILE <= kSegmentMaxTiles) {
+    const uint32_t sm = segment_smem(head_dim);
+    int o16 = 0, o_bf = 0;
+    if ((rc = blocks_per_sm(segment_kernel_for(PA_FLOAT16, head_dim, G), sm, &o16)) != PA_OK) return rc;
+    if ((rc = blocks_per_sm(segment_kernel_for(PA_BFLOAT16, head_dim, G), sm, &o_bf)) != PA_OK) return rc;
+    if ((long long)num_seqs * num_kv_heads * (group / G) <= (long long)sms * std::min(o16, o_bf)) {
+      lp->segment_mode = true;
+      lp->smem = sm;
+      lp->grid = num_seqs * num_kv_heads * (group / G);
+      lp->chunk_tiles = 0;
+      lp->max_chunks = 0;
+      lp->queue_bytes = lp->tiles_bytes = lp->ml_bytes = lp->acc_bytes = lp->total_bytes = 0;
+      return PA_OK;
+    }
+  }
   lp->smem = split_smem(head_dim, group, num_seqs);
   if (lp->smem > 227u * 1024u) return PA_ERR_SHAPE;
   int occ_f16 = 0, occ_bf16 = 0;
@@ -275,8 +317,11 @@ int plan_decode(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, i
   return PA_OK;
 }
 
-// ---- TMA tensor maps of the caches, viewed as [num_blocks * num_kv_heads * block_size rows][head_dim],
-// boxes of 16 rows x 64 elements (128 bytes) with the 128-byte swizzle.
+// ---- TMA tensor maps of the caches, with the 128-byte swizzle.  2-D (prefill): the cache viewed as
+// [num_blocks * num_kv_heads * block_size rows][head_dim], boxes of 16 rows x 64 elements (128 bytes).
+// 3-D (decode): the same rows with each row's 64-element halves as a third dimension 128 bytes apart, so
+// that one box brings a whole 16-row tile stored as [halves][16 rows][128 bytes]: one copy per K or V
+// tile instead of one per half (measured: 43.0 against 44.7 us per call on the shared-prefix step).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder(int *rc) {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -300,8 +345,10 @@ struct MapKey {
   const void *base;
   long long rows;
   int head_dim, dtype;
+  bool three_d;
   bool operator==(const MapKey &o) const {
-    return dev == o.dev && base == o.base && rows == o.rows && head_dim == o.head_dim && dtype == o.dtype;
+    return dev == o.dev && base == o.base && rows == o.rows && head_dim == o.head_dim && dtype == o.dtype &&
+           three_d == o.three_d;
   }
 };
 struct MapEntry {
@@ -312,11 +359,11 @@ struct MapEntry {
 MapEntry g_maps[32];
 int g_map_next = 0;
 
-int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, CUtensorMap *out) {
+int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, bool three_d, CUtensorMap *out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record(e);
-  const MapKey key{dev, base, rows, head_dim, dtype};
+  const MapKey key{dev, base, rows, head_dim, dtype, three_d};
   std::lock_guard<std::mutex> lk(g_mu);
   for (auto &m : g_maps)
     if (m.used && m.key == key) {
@@ -327,12 +374,25 @@ int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, 
   auto encode = tensor_map_encoder(&rc);
   if (!encode) return rc;
   CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)pa::TILE};
-  const cuuint32_t elem_strides[2] = {1, 1};
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  cuuint32_t rank;
+  if (three_d) {
+    // [halves][rows][64 elements]: x = element in a half, y = row (head_dim * 2 bytes apart), z = half
+    // (128 bytes apart); one box covers a 16-row tile of both halves
+    dims[0] = 64, dims[1] = (cuuint64_t)rows, dims[2] = (cuuint64_t)head_dim / 64;
+    strides[0] = (cuuint64_t)head_dim * 2, strides[1] = 128;
+    box[0] = 64, box[1] = (cuuint32_t)pa::TILE, box[2] = (cuuint32_t)head_dim / 64;
+    rank = 3;
+  } else {
+    dims[0] = (cuuint64_t)head_dim, dims[1] = (cuuint64_t)rows;
+    strides[0] = (cuuint64_t)head_dim * 2;
+    box[0] = 64, box[1] = (cuuint32_t)pa::TILE;
+    rank = 2;
+  }
   const CUresult r =
-      encode(&map, dtype == PA_BFLOAT16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+      encode(&map, dtype == PA_BFLOAT16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank,
              const_cast<void *>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -348,13 +408,25 @@ int cache_tensor_map(const void *base, long long rows, int head_dim, int dtype, 
 template <class E, int D>
 int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype, cudaStream_t stream) {
   const int threads = kWarps * 32;
+  if (lp.segment_mode) {
+    cudaError_t e = args.heads_per_unit == 2
+                        ? launch_pdl(pa::decode_segment_kernel<E, D, 2, kWarps, kStages>, dim3(lp.grid),
+                                     dim3(threads), lp.smem, stream, args)
+                        : launch_pdl(pa::decode_segment_kernel<E, D, 1, kWarps, kStages>, dim3(lp.grid),
+                                     dim3(threads), lp.smem, stream, args);
+    if (e != cudaSuccess) return record(e);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return record(e);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return PA_OK;
+  }
   if (uses_mma(args.group)) {
     const long long rows = args.num_blocks * args.num_kv_heads * args.block_size;
     if (rows > 0x7fffffffLL) return PA_ERR_SHAPE;  // TMA coordinates are signed 32-bit
     CUtensorMap mk, mv;
-    int rc = cache_tensor_map(args.k_cache, rows, D, dtype, &mk);
+    int rc = cache_tensor_map(args.k_cache, rows, D, dtype, true, &mk);
     if (rc != PA_OK) return rc;
-    rc = cache_tensor_map(args.v_cache, rows, D, dtype, &mv);
+    rc = cache_tensor_map(args.v_cache, rows, D, dtype, true, &mv);
     if (rc != PA_OK) return rc;
     cudaError_t e = launch_pdl(pa::decode_split_mma_kernel<E, D, kWarps, kStages>, dim3(lp.grid), dim3(threads),
                                lp.smem, stream, mk, mv, args);
@@ -372,7 +444,11 @@ int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype,
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   // merge: one warp per query head on the tensor-core path (segments of 3 to 8 heads), one warp per segment
-  // (1 or 2 heads) on the CUDA-core path; eight warps per block
+  // (1 or 2 heads) on the CUDA-core path; eight warps per block.  Measured and dropped: merging in the
+  // tensor-core split kernel itself (the warp that stores a segment's last cut piece merges it, counted
+  // through per-segment arrival words): 179 against 167 us on the 32 query / 8 kv head batch and 62
+  // against 43 us on the shared-prefix step -- the merges then run one after another at the end of each
+  // warp's stream instead of in parallel across the merge grid.
   const int hw = uses_mma(args.group) ? 1 : args.heads_per_unit;
   const long long warps = (long long)args.num_seqs * args.num_kv_heads * args.n_chunks * (args.heads_per_unit / hw);
   const dim3 mgrid((unsigned)((warps + 7) / 8)), mblock(256);
@@ -491,7 +567,8 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   LaunchPlan lp;
   rc = plan_decode(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, dtype, &lp);
   if (rc != PA_OK) return rc;
-  if (!workspace || workspace_bytes < lp.total_bytes || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+  if (lp.total_bytes > 0 && (!workspace || workspace_bytes < lp.total_bytes || !aligned16(workspace)))
+    return PA_ERR_WORKSPACE;
 
   const int group = num_q_heads / num_kv_heads;
   const int G = heads_per_unit(group);
@@ -503,10 +580,17 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.out = static_cast<uint16_t *>(out);
-  a.ws_queue = reinterpret_cast<unsigned long long *>(ws);
-  a.ws_tiles = reinterpret_cast<int *>(ws + lp.queue_bytes);
-  a.ws_ml = reinterpret_cast<float2 *>(ws + lp.queue_bytes + lp.tiles_bytes);
-  a.ws_acc = reinterpret_cast<float *>(ws + lp.queue_bytes + lp.tiles_bytes + lp.ml_bytes);
+  if (lp.segment_mode) {  // no workspace
+    a.ws_queue = nullptr;
+    a.ws_tiles = nullptr;
+    a.ws_ml = nullptr;
+    a.ws_acc = nullptr;
+  } else {
+    a.ws_queue = reinterpret_cast<unsigned long long *>(ws);
+    a.ws_tiles = reinterpret_cast<int *>(ws + lp.queue_bytes);
+    a.ws_ml = reinterpret_cast<float2 *>(ws + lp.queue_bytes + lp.tiles_bytes);
+    a.ws_acc = reinterpret_cast<float *>(ws + lp.queue_bytes + lp.tiles_bytes + lp.ml_bytes);
+  }
   a.num_blocks = num_blocks;
   a.q_seq_stride = q_seq_stride;
   a.out_seq_stride = out_seq_stride;
@@ -719,9 +803,9 @@ int pa_prefill(const void *q, const void *k_cache, const void *v_cache, const in
       return PA_ERR_CUDA;
     }
   }
-  rc = cache_tensor_map(k_cache, rows, head_dim, dtype, &mk);
+  rc = cache_tensor_map(k_cache, rows, head_dim, dtype, false, &mk);
   if (rc != PA_OK) return rc;
-  rc = cache_tensor_map(v_cache, rows, head_dim, dtype, &mv);
+  rc = cache_tensor_map(v_cache, rows, head_dim, dtype, false, &mv);
   if (rc != PA_OK) return rc;
 
   pa::PrefillArgs a;

@@ -349,30 +349,32 @@ __device__ __forceinline__ int chunk_first_head(const DecodeArgs &a, int hc) {
 // slot is flagged in `bad_slots`.
 struct TileProducer {
   TilePos pos;
-  int win_s, win_base, win_nblk, ent;
-  uint32_t bad_slots;
+  int win_s, win_base, ent;  // the table window in use: entries [win_base, win_base + 32) of row win_s
+  uint32_t bad_slots;        // ring slots whose tile was not copied (set or cleared at every issue)
 
-  __device__ __forceinline__ void start(const TilePos &p) {
-    pos = p;
+  __device__ __forceinline__ void init() {
     win_s = -1;
     win_base = 0;
-    win_nblk = 0;
     ent = -1;
     bad_slots = 0;
   }
 
+  // Moves the producer to a new position.  The window stays valid (it depends on the table row only), and
+  // so do the flags of the slots still in flight from the previous chunk.
+  __device__ __forceinline__ void start(const TilePos &p) { pos = p; }
+
   // Returns the physical block of the producer's current tile (or -1), loading a new window when needed.
+  // The row's block count comes from the sequence's tile count nt = ceil(L / 16)
+  // (ceil(nt * 16 / block_size) = ceil(L / block_size)), so no length load stands between the producer and
+  // the table; entries at or past it are not read.
   __device__ __forceinline__ int lookup(const DecodeArgs &a, int lane) {
     const int blk = (pos.j * TILE) / a.block_size;
     if (pos.s != win_s || blk < win_base || blk >= win_base + 32) {
-      if (pos.s != win_s) {
-        win_s = pos.s;
-        const int L = __ldg(a.context_lens + pos.s);
-        win_nblk = (L + a.block_size - 1) / a.block_size;
-      }
+      win_s = pos.s;
       win_base = blk & ~31;
-      const bool in_row = dcheck(pos.s < a.num_seqs && win_nblk <= a.table_stride);
-      ent = (in_row && win_base + lane < win_nblk)
+      const int nblk = (pos.nt * TILE + a.block_size - 1) / a.block_size;
+      const bool in_row = dcheck(pos.s < a.num_seqs && nblk <= a.table_stride);
+      ent = (in_row && win_base + lane < nblk)
                 ? __ldg(a.block_tables + (long long)pos.s * a.table_stride + win_base + lane)
                 : -1;
     }
@@ -463,26 +465,158 @@ __device__ __forceinline__ bool wait_slot(uint64_t *bars, uint32_t it, int in_fl
   return false;
 }
 
+constexpr float RESCALE_SLACK = 8.f;
+
+// The arithmetic of the CUDA-core kernels for one piece (a run of tiles of one segment: G query heads of
+// one kv head), shared by the split and the per-segment kernels: the query rows, the online-softmax state
+// and accumulators, and the step for one 16-token tile.
+//
+// Per tile, lane l holds 16 bytes (8 head dims, cl * 8 ..) of rows r * NGRP + grp (r < R) of K and of V.
+// QK^T uses the mixed-precision fma (2-byte inputs, fp32 accumulation); the 16 dot products are finished
+// by a reduce-scatter butterfly.  The online softmax keeps, per query head, a running maximum m that is
+// raised only when a logit exceeds it by more than RESCALE_SLACK (base-2 units), so most tiles need no max
+// reduction; m cancels between numerator and denominator, and weights stay below 2^RESCALE_SLACK.
+template <class E, int D, int G>
+struct CoreMath {
+  static constexpr int LPR = D / 8;      // lanes covering one K/V row
+  static constexpr int NGRP = 32 / LPR;  // rows one warp-wide 16-byte load covers
+  static constexpr int R = TILE / NGRP;  // rows per lane per tile
+  int grp, cl, my_tok;
+  uint32_t qw[G][4];
+  float m[G], lsum[G];
+  float2 acc[G][4];
+
+  __device__ __forceinline__ void setup(int lane) {
+    grp = lane / LPR;
+    cl = lane % LPR;
+    my_tok = ((lane & (LPR - 2)) >> 1) * NGRP + grp;  // token whose logit this lane ends with
+  }
+
+  // A new piece: the G query rows starting at qrow (D elements apart), zeros when !ok; a fresh state.
+  __device__ __forceinline__ void begin(const uint16_t *qrow, bool ok) {
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      const uint4 w = ok ? __ldg(reinterpret_cast<const uint4 *>(qrow + gg * D + cl * 8)) : make_uint4(0, 0, 0, 0);
+      qw[gg][0] = w.x;
+      qw[gg][1] = w.y;
+      qw[gg][2] = w.z;
+      qw[gg][3] = w.w;
+      m[gg] = -INFINITY;
+      lsum[gg] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) acc[gg][kk] = make_float2(0.f, 0.f);
+    }
+  }
+
+  // This lane's rows of the K tile at kt and the V tile at vt (zeros for a tile that was not copied).
+  __device__ __forceinline__ void read_tile(const unsigned char *kt, const unsigned char *vt, bool bad, uint4 (&kr)[R],
+                                            uint4 (&vr)[R]) const {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      kr[r] = bad ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4 *>(kt + ((r * NGRP + grp) * D + cl * 8) * 2);
+      vr[r] = bad ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4 *>(vt + ((r * NGRP + grp) * D + cl * 8) * 2);
+    }
+  }
+
+  // One tile of nvalid live rows (the rest masked): QK^T, scale, mask, online softmax, P.V.
+  __device__ __forceinline__ void tile(const uint4 (&kr)[R], const uint4 (&vr)[R], int nvalid, float scale_log2,
+                                       int lane) {
+    const bool tok_live = my_tok < nvalid;
+    // QK^T for this lane's R rows, the butterfly, scale, mask
+    float z[G];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      float part[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) part[r] = E::dot8(qw[gg], kr[r], 0.f);
+      const float t = row_group_reduce<R>(part, lane) * scale_log2;
+      z[gg] = tok_live ? t : -INFINITY;
+    }
+    // softmax state: raise m only when some logit passes it by more than the slack
+    float pr[G][R];
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      if (__any_sync(FULL, z[gg] > m[gg] + RESCALE_SLACK)) {
+        float mt = z[gg];
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 4));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
+        const float alpha = exp2f(m[gg] - mt);  // 0 on the piece's first tile (m = -inf)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) acc[gg][kk] = make_float2(acc[gg][kk].x * alpha, acc[gg][kk].y * alpha);
+        lsum[gg] *= alpha;
+        m[gg] = mt;
+      }
+      const float pz = exp2f(z[gg] - m[gg]);
+      lsum[gg] += (lane & 1) ? 0.f : pz;
+#pragma unroll
+      for (int r = 0; r < R; ++r) pr[gg][r] = __shfl_sync(FULL, pz, grp * LPR + 2 * r);
+    }
+    // P.V over this lane's 8 dims and R rows (packed fp32 fma)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float vf[8];
+      E::widen8(vr[r], vf);
+      if (nvalid < TILE) {  // rows past the sequence may hold anything (NaN): never let them in
+        const bool row_live = (r * NGRP + grp) < nvalid;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) vf[kk] = row_live ? vf[kk] : 0.f;
+      }
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        const float2 pp = make_float2(pr[gg][r], pr[gg][r]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) acc[gg][kk] = __ffma2_rn(pp, make_float2(vf[2 * kk], vf[2 * kk + 1]), acc[gg][kk]);
+      }
+    }
+  }
+
+  // End of the piece: merges the row groups (lanes < LPR then hold dims cl * 8 .. cl * 8 + 7 of every head,
+  // un-normalised) and totals the sums in every lane.
+  __device__ __forceinline__ void finish() {
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+#pragma unroll
+      for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          acc[gg][kk].x += __shfl_xor_sync(FULL, acc[gg][kk].x, off);
+          acc[gg][kk].y += __shfl_xor_sync(FULL, acc[gg][kk].y, off);
+        }
+      }
+      float l = lsum[gg];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
+      lsum[gg] = l;
+    }
+  }
+
+  // Lanes < LPR: the normalised rows (zeros when bad) of the G heads, heads D elements apart from out_row.
+  __device__ __forceinline__ void store_output(uint16_t *out_row, bool bad) const {
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      float o[8];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        o[2 * kk] = bad ? 0.f : acc[gg][kk].x / lsum[gg];
+        o[2 * kk + 1] = bad ? 0.f : acc[gg][kk].y / lsum[gg];
+      }
+      *reinterpret_cast<uint4 *>(out_row + gg * D + cl * 8) = narrow8<E>(o);
+    }
+  }
+};
+
 // CUDA-core split kernel, for head chunks of G = 1 or 2 query heads.
 //
 // Each warp streams the tiles of its chunks through a private STAGES-deep ring
 // of shared-memory slots filled by bulk copies (K tile + V tile of one
-// (block, kv head), 2 x 16 * D * 2 bytes).  Per tile, lane l copies 16 bytes
-// (8 head dims) of rows r*NGRP + l/LPR (r < R) of K and of V from the slot
-// into registers and the slot is refilled at once, before the math.  QK^T uses
-// the mixed-precision fma (2-byte inputs, fp32 accumulation); the 16 dot
-// products are finished by a reduce-scatter butterfly.  The online softmax
-// keeps, per query head, a running maximum m that is raised only when a logit
-// exceeds it by more than RESCALE_SLACK (base-2 units), so most tiles need no
-// max reduction; m cancels between numerator and denominator, and weights
-// stay below 2^RESCALE_SLACK.
-constexpr float RESCALE_SLACK = 8.f;
-
+// (block, kv head), 2 x 16 * D * 2 bytes).  Per tile, each lane copies its
+// rows of K and V from the slot into registers and the slot is refilled at
+// once, before the math (CoreMath).
 template <class E, int D, int G, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(const DecodeArgs a) {
-  constexpr int LPR = D / 8;       // lanes covering one K/V row
-  constexpr int NGRP = 32 / LPR;   // rows one warp-wide 16-byte load covers
-  constexpr int R = TILE / NGRP;   // rows per lane per tile
+  constexpr int LPR = CoreMath<E, D, G>::LPR;
   constexpr uint32_t TILE_BYTES = TILE * D * 2;
   constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;
   using Smem = SplitSmem<WARPS, STAGES, STAGE_BYTES>;
@@ -508,9 +642,6 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
   const ChunkPlan plan = plan_chunks(a, pt[S]);
   const int HC = a.num_kv_heads * a.n_chunks;
 
-  const int grp = lane / LPR;
-  const int cl = lane % LPR;
-  const int my_tok = ((lane & (LPR - 2)) >> 1) * NGRP + grp;  // token whose logit this lane ends with
   uint32_t iter = 0;  // tiles consumed by this warp: ring slot iter % STAGES, phase (iter / STAGES) & 1
   TileProducer prod;
 
@@ -522,6 +653,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
     int prod_left = plan.length(prod_c);
     bool prod_done = false;
     TilePos cp = locate_tile(pt, S, HC, plan.start(cons_c));
+    prod.init();
     prod.start(cp);
     uint32_t issued = iter;  // tiles issued by this warp: the next goes to ring slot issued % STAGES
 
@@ -565,9 +697,8 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
     };
     for (int k = 0; k < STAGES; ++k) issue_next();
 
-    uint32_t qw[G][4];
-    float m[G], lsum[G];
-    float2 acc[G][4];
+    CoreMath<E, D, G> cm;
+    cm.setup(lane);
     int L = 0, hq0 = 0, slot = 0;
     bool full = false, piece_bad = false;
 
@@ -589,126 +720,27 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
         const bool q_ok = dcheck(cp.s < S && hq0 + G <= a.num_q_heads);
         L = q_ok ? __ldg(a.context_lens + cp.s) : 0;
         piece_bad = false;
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          const uint4 w = q_ok ? __ldg(reinterpret_cast<const uint4 *>(a.q + (long long)cp.s * a.q_seq_stride +
-                                                                       (long long)(hq0 + gg) * D + cl * 8))
-                               : make_uint4(0, 0, 0, 0);
-          qw[gg][0] = w.x;
-          qw[gg][1] = w.y;
-          qw[gg][2] = w.z;
-          qw[gg][3] = w.w;
-          m[gg] = -INFINITY;
-          lsum[gg] = 0.f;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) acc[gg][kk] = make_float2(0.f, 0.f);
-        }
+        cm.begin(a.q + (long long)cp.s * a.q_seq_stride + (long long)hq0 * D, q_ok);
       }
       const int st = (int)(iter % STAGES);
       if (!wait_slot<STAGES>(bars, iter, (int)(issued - iter), a.wait_limit_ns, lane)) return;
       const bool tile_bad = (prod.bad_slots >> st) & 1u;
       // copy this lane's rows out of the slot, then hand the slot straight back to the copy engine
-      const unsigned char *kt = ring + st * STAGE_BYTES;
-      const unsigned char *vt = kt + TILE_BYTES;
-      uint4 kr[R], vr[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        kr[r] = tile_bad ? make_uint4(0, 0, 0, 0)
-                         : *reinterpret_cast<const uint4 *>(kt + ((r * NGRP + grp) * D + cl * 8) * 2);
-        vr[r] = tile_bad ? make_uint4(0, 0, 0, 0)
-                         : *reinterpret_cast<const uint4 *>(vt + ((r * NGRP + grp) * D + cl * 8) * 2);
-      }
+      uint4 kr[CoreMath<E, D, G>::R], vr[CoreMath<E, D, G>::R];
+      cm.read_tile(ring + st * STAGE_BYTES, ring + st * STAGE_BYTES + TILE_BYTES, tile_bad, kr, vr);
       __syncwarp();
       issue_next();
       ++iter;
       piece_bad |= tile_bad;
-
-      if (!piece_bad) {
-        const int nvalid = min(TILE, L - cp.j * TILE);
-        const bool tok_live = my_tok < nvalid;
-        // QK^T for this lane's R rows, the butterfly, scale, mask
-        float z[G];
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          float part[R];
-#pragma unroll
-          for (int r = 0; r < R; ++r) part[r] = E::dot8(qw[gg], kr[r], 0.f);
-          const float t = row_group_reduce<R>(part, lane) * a.scale_log2;
-          z[gg] = tok_live ? t : -INFINITY;
-        }
-        // softmax state: raise m only when some logit passes it by more than the slack
-        float pr[G][R];
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-          if (__any_sync(FULL, z[gg] > m[gg] + RESCALE_SLACK)) {
-            float mt = z[gg];
-            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
-            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 4));
-            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
-            mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
-            const float alpha = exp2f(m[gg] - mt);  // 0 on the piece's first tile (m = -inf)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) acc[gg][kk] = make_float2(acc[gg][kk].x * alpha, acc[gg][kk].y * alpha);
-            lsum[gg] *= alpha;
-            m[gg] = mt;
-          }
-          const float pz = exp2f(z[gg] - m[gg]);
-          lsum[gg] += (lane & 1) ? 0.f : pz;
-#pragma unroll
-          for (int r = 0; r < R; ++r) pr[gg][r] = __shfl_sync(FULL, pz, grp * LPR + 2 * r);
-        }
-        // P.V over this lane's 8 dims and R rows (packed fp32 fma)
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          float vf[8];
-          E::widen8(vr[r], vf);
-          if (nvalid < TILE) {  // rows past the sequence may hold anything (NaN): never let them in
-            const bool row_live = (r * NGRP + grp) < nvalid;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) vf[kk] = row_live ? vf[kk] : 0.f;
-          }
-#pragma unroll
-          for (int gg = 0; gg < G; ++gg) {
-            const float2 pp = make_float2(pr[gg][r], pr[gg][r]);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              acc[gg][kk] = __ffma2_rn(pp, make_float2(vf[2 * kk], vf[2 * kk + 1]), acc[gg][kk]);
-          }
-        }
-      }
+      if (!piece_bad) cm.tile(kr, vr, min(TILE, L - cp.j * TILE), a.scale_log2, lane);
 
       if (cp.j + 1 == cp.nt || cons_left == 1) {
         // ---- end of the piece: merge the row groups, total the sums, store the output or the partial
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg) {
-#pragma unroll
-          for (int off = LPR; off < 32; off <<= 1) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              acc[gg][kk].x += __shfl_xor_sync(FULL, acc[gg][kk].x, off);
-              acc[gg][kk].y += __shfl_xor_sync(FULL, acc[gg][kk].y, off);
-            }
-          }
-          float l = lsum[gg];
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
-          lsum[gg] = l;
-        }
+        cm.finish();
         if (piece_bad && lane == 0) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
         if (full) {
-          if (lane < LPR && dcheck(cp.s < S && hq0 + G <= a.num_q_heads)) {
-            uint16_t *out_row = a.out + (long long)cp.s * a.out_seq_stride + (long long)hq0 * D + cl * 8;
-#pragma unroll
-            for (int gg = 0; gg < G; ++gg) {
-              float o[8];
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                o[2 * kk] = piece_bad ? 0.f : acc[gg][kk].x / lsum[gg];
-                o[2 * kk + 1] = piece_bad ? 0.f : acc[gg][kk].y / lsum[gg];
-              }
-              *reinterpret_cast<uint4 *>(out_row + gg * D) = narrow8<E>(o);
-            }
-          }
+          if (lane < LPR && dcheck(cp.s < S && hq0 + G <= a.num_q_heads))
+            cm.store_output(a.out + (long long)cp.s * a.out_seq_stride + (long long)hq0 * D, piece_bad);
         } else {
           const long long prow = (cons_c * 2 + slot) * G;
           const bool row_ok = dcheck(cons_c < a.max_chunks);
@@ -716,17 +748,165 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
           for (int gg = 0; gg < G; ++gg) {
             if (!row_ok) break;
             if (lane < LPR && !piece_bad) {
-              float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + (prow + gg) * D + cl * 8);
-              dst[0] = make_float4(acc[gg][0].x, acc[gg][0].y, acc[gg][1].x, acc[gg][1].y);
-              dst[1] = make_float4(acc[gg][2].x, acc[gg][2].y, acc[gg][3].x, acc[gg][3].y);
+              float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + (prow + gg) * D + cm.cl * 8);
+              dst[0] = make_float4(cm.acc[gg][0].x, cm.acc[gg][0].y, cm.acc[gg][1].x, cm.acc[gg][1].y);
+              dst[1] = make_float4(cm.acc[gg][2].x, cm.acc[gg][2].y, cm.acc[gg][3].x, cm.acc[gg][3].y);
             }
-            if (lane == 0) a.ws_ml[prow + gg] = piece_bad ? make_float2(-INFINITY, -1.f) : make_float2(m[gg], lsum[gg]);
+            if (lane == 0)
+              a.ws_ml[prow + gg] = piece_bad ? make_float2(-INFINITY, -1.f) : make_float2(cm.m[gg], cm.lsum[gg]);
           }
         }
       }
       advance_tile(cp, pt, S, HC);
       --cons_left;
       ++k;
+    }
+  }
+}
+
+// Per-segment kernel for small batches on the CUDA-core path: block b handles segment b (sequence
+// s = b / HC, head chunk hc = b % HC) whole.  Its WARPS warps take the segment's tiles in turn (tile j to
+// warp j mod WARPS), each through its own ring of bulk copies as in the split kernel; at the end the warps'
+// softmax states are merged in shared memory, in warp order (deterministic), and warp 0 writes the rows.
+// It needs no workspace and no merge kernel, and a block touches only its own sequence's length and table
+// row: chosen when all segments fit one wave of blocks and are short, where the split kernel's tile
+// prefix, chunk queue and separate merge launch would cost more than the work.
+template <class E, int D, int G, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32) decode_segment_kernel(const DecodeArgs a) {
+  using CM = CoreMath<E, D, G>;
+  constexpr int LPR = CM::LPR;
+  constexpr uint32_t TILE_BYTES = TILE * D * 2;
+  constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;
+  using Smem = SplitSmem<WARPS, STAGES, STAGE_BYTES>;
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  unsigned char *ring = smem + warp * STAGES * STAGE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Smem::RING) + warp * STAGES;
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bars[st], 1);
+    fence_mbar_init();
+  }
+  grid_dependency_wait();  // every input may come from the previous kernel in the stream
+  grid_launch_dependents();
+  const int HC = a.num_kv_heads * a.n_chunks;
+  const int s = (int)(blockIdx.x / HC), hc = (int)(blockIdx.x - (unsigned)s * HC);
+  const int hq0 = chunk_first_head(a, hc);
+  const int h = hc / a.n_chunks;
+  const int L = __ldg(a.context_lens + s);
+  uint16_t *out_row = a.out + (long long)s * a.out_seq_stride + (long long)hq0 * D;
+  if (!context_ok(a, L) || L == 0) {  // zero rows; the status bit once per sequence
+    if (warp == 0) {
+      if (lane == 0 && L != 0 && hc == 0)
+        atomicOr(&g_status, (L < 0 || (long long)L > (long long)a.table_stride * a.block_size) ? PA_DEV_ERR_CONTEXT
+                                                                                              : PA_DEV_ERR_CONTEXT_HINT);
+      for (int c = lane; c < G * D / 8; c += 32) reinterpret_cast<uint4 *>(out_row)[c] = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
+  const int nt = (L + TILE - 1) / TILE;
+  const int nblk = (L + a.block_size - 1) / a.block_size;
+  const int my_tiles = warp < nt ? (nt - warp + WARPS - 1) / WARPS : 0;
+
+  // physical block of tile j, through a 32-entry window of the table row (entries >= nblk not read)
+  int win_base = -1, ent = -1;
+  auto phys_of = [&](int j) -> int {
+    const int blk = (j * TILE) / a.block_size;
+    const int base = blk & ~31;
+    if (base != win_base) {
+      win_base = base;
+      ent = (base + lane < nblk && dcheck(nblk <= a.table_stride))
+                ? __ldg(a.block_tables + (long long)s * a.table_stride + base + lane)
+                : -1;
+    }
+    const int phys = __shfl_sync(FULL, ent, blk - base);
+    return (phys >= 0 && (long long)phys < a.num_blocks) ? phys : -1;
+  };
+  uint32_t bad_slots = 0;
+  auto issue = [&](int t) {  // this warp's t-th tile into slot t % STAGES
+    const int j = warp + t * WARPS;
+    const int phys = phys_of(j);
+    const int st = t % STAGES;
+    bad_slots = phys >= 0 ? (bad_slots & ~(1u << st)) : (bad_slots | (1u << st));
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      if (phys >= 0) {
+        const long long row0 = ((long long)phys * a.num_kv_heads + h) * a.block_size + (j * TILE) % a.block_size;
+        unsigned char *dst = ring + st * STAGE_BYTES;
+        mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
+        bulk_copy_g2s(dst, a.k_cache + row0 * D, TILE_BYTES, &bars[st]);
+        bulk_copy_g2s(dst + TILE_BYTES, a.v_cache + row0 * D, TILE_BYTES, &bars[st]);
+      } else {
+        mbar_arrive(&bars[st]);
+      }
+    }
+  };
+
+  CM cm;
+  cm.setup(lane);
+  cm.begin(a.q + (long long)s * a.q_seq_stride + (long long)hq0 * D, true);
+  int issued = 0;
+  for (; issued < STAGES && issued < my_tiles; ++issued) issue(issued);
+  bool bad = false;
+  for (int t = 0; t < my_tiles; ++t) {
+    const int st = t % STAGES;
+    if (!wait_slot<STAGES>(bars, (uint32_t)t, issued - t, a.wait_limit_ns, lane)) {
+      bad = true;  // timed out (flagged; the copies in flight were waited for): this segment's rows become zeros
+      break;
+    }
+    uint4 kr[CM::R], vr[CM::R];
+    const bool tile_bad = (bad_slots >> st) & 1u;
+    cm.read_tile(ring + st * STAGE_BYTES, ring + st * STAGE_BYTES + TILE_BYTES, tile_bad, kr, vr);
+    __syncwarp();
+    if (issued < my_tiles) issue(issued++);
+    bad |= tile_bad;
+    const int j = warp + t * WARPS;
+    if (!bad) cm.tile(kr, vr, min(TILE, L - j * TILE), a.scale_log2, lane);
+  }
+  cm.finish();
+
+  // merge the warps' states through shared memory (the rings are free: every copy issued was waited for)
+  __syncthreads();
+  float *x_acc = reinterpret_cast<float *>(smem);                  // [WARPS][G][D]
+  float2 *x_ml = reinterpret_cast<float2 *>(x_acc + WARPS * G * D);  // [WARPS][G]
+  int *x_bad = reinterpret_cast<int *>(x_ml + WARPS * G);          // [WARPS]
+#pragma unroll
+  for (int gg = 0; gg < G; ++gg) {
+    if (lane < LPR) {
+      float4 *dst = reinterpret_cast<float4 *>(x_acc + (warp * G + gg) * D + cm.cl * 8);
+      dst[0] = make_float4(cm.acc[gg][0].x, cm.acc[gg][0].y, cm.acc[gg][1].x, cm.acc[gg][1].y);
+      dst[1] = make_float4(cm.acc[gg][2].x, cm.acc[gg][2].y, cm.acc[gg][3].x, cm.acc[gg][3].y);
+    }
+    if (lane == 0) x_ml[warp * G + gg] = make_float2(cm.m[gg], cm.lsum[gg]);
+  }
+  if (lane == 0) x_bad[warp] = bad ? 1 : 0;
+  __syncthreads();
+  if (warp != 0) return;
+  bool any_bad = false;
+#pragma unroll
+  for (int w = 0; w < WARPS; ++w) any_bad |= x_bad[w] != 0;
+  if (any_bad && lane == 0) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
+  if (lane < LPR) {
+#pragma unroll
+    for (int gg = 0; gg < G; ++gg) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < WARPS; ++w) M = fmaxf(M, x_ml[w * G + gg].x);
+      float l = 0.f, o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int w = 0; w < WARPS; ++w) {
+        const float2 ml = x_ml[w * G + gg];
+        const float wt = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;  // a warp with no tiles has m = -inf, l = 0
+        l = fmaf(ml.y, wt, l);
+        const float *src = x_acc + (w * G + gg) * D + cm.cl * 8;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) o[kk] = fmaf(wt, src[kk], o[kk]);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) o[kk] = any_bad ? 0.f : o[kk] / l;
+      *reinterpret_cast<uint4 *>(out_row + gg * D + cm.cl * 8) = narrow8<E>(o);
     }
   }
 }

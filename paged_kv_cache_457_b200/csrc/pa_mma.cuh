@@ -5,8 +5,10 @@
 // Per 16-token tile, with the unit's query heads as the N = 8 columns:
 //   S^T[16 tokens x 8 heads]  = K[16 x d] . Q^T[d x 8]          (d/16 mma)
 //   O^T[d x 8 heads]         += V^T[d x 16 tokens] . P^T[16 x 8] (2 * d/16 mma)
-// K and V tiles arrive by 2-D TMA tensor copies with the 128-byte swizzle, so
-// the ldmatrix loads of both operands are free of bank conflicts.  P is
+// K and V tiles arrive by TMA tensor copies with the 128-byte swizzle (one
+// 3-D box per tile: the D / 64 halves of the 16 rows, each stored as 16 rows
+// of 128 bytes), so the ldmatrix loads of both operands are free of bank
+// conflicts.  P is
 // split into a 2-byte head and a 2-byte residual (P ~= Ph + Pl, relative
 // error ~2^-16) so the product keeps fp32-level accuracy although the mma
 // takes 2-byte operands; movmatrix turns P^T's accumulator layout into the
@@ -17,6 +19,7 @@
 #include <cuda.h>
 
 #include "pa_kernels.cuh"
+#include "pa_tcgen05.cuh"
 
 namespace pa {
 
@@ -80,7 +83,6 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
     decode_split_mma_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                             const DecodeArgs a) {
   constexpr int KSTEPS = D / 16;  // 16-dim steps of QK^T, and 16-dim row tiles of O^T
-  constexpr int BOXES = D / 64;
   constexpr uint32_t TILE_BYTES = TILE * D * 2;
   using Smem = MmaSmem<E, D, WARPS, STAGES>;
   constexpr uint32_t STAGE_BYTES = Smem::STAGE_BYTES;
@@ -129,6 +131,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
     int prod_left = plan.length(prod_c);
     bool prod_done = false;
     TilePos cp = locate_tile(pt, S, HC, plan.start(cons_c));
+    prod.init();
     prod.start(cp);
     uint32_t issued = iter;  // tiles issued by this warp: the next goes to ring slot issued % STAGES
 
@@ -151,17 +154,15 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
       const int phys = prod.lookup(a, lane);
       const int st = (int)(it % STAGES);
       prod.bad_slots = phys >= 0 ? (prod.bad_slots & ~(1u << st)) : (prod.bad_slots | (1u << st));
+      // one 3-D box per K and per V tile: [D / 64 halves][16 rows][64 elements] (see cache_tensor_map)
       if (lane == 0) {
         fence_proxy_async_smem();
         if (phys >= 0) {
           const int row0 = (int)prod.first_row(a, phys);  // lookup() checked the tile lies in its slab
           unsigned char *dst = ring + st * STAGE_BYTES;
           mbar_arrive_expect_tx(&bars[st], STAGE_BYTES);
-#pragma unroll
-          for (int bx = 0; bx < BOXES; ++bx) {
-            tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, row0, &bars[st]);
-            tma_load_2d(dst + TILE_BYTES + bx * 2048, &tmap_v, bx * 64, row0, &bars[st]);
-          }
+          tc::tma_load_3d(dst, &tmap_k, 0, row0, 0, &bars[st]);
+          tc::tma_load_3d(dst + TILE_BYTES, &tmap_v, 0, row0, 0, &bars[st]);
         } else {
           mbar_arrive(&bars[st]);
         }

@@ -100,3 +100,65 @@ def test_small_shapes(hq, hkv, d, bs, dtype, partition):
     out = dev.decode(st, partition_tokens=partition)
     _, _, ref = oracle_step(wl, wl.k_cache, wl.v_cache, st)
     compare(out, ref, dtype, what=f"{hq}/{hkv} d{d} bs{bs} {dtype} part {partition}")
+
+
+SEGMENT_SHAPES = [  # (hq, hkv, d, bs, dtype): CUDA-core groups of 1 and 2 heads
+    (8, 8, 64, 16, "fp16"),
+    (8, 8, 128, 32, "bf16"),
+    (8, 4, 128, 16, "bf16"),
+    (4, 2, 64, 32, "fp16"),
+]
+SEGMENT_LENS = [0, 1, 2, 15, 16, 17, 31, 33, 100, 255, 256, 257, 400, 511, 512]
+
+
+@pytest.mark.parametrize("hq,hkv,d,bs,dtype", SEGMENT_SHAPES)
+def test_small_batch_segment_path(hq, hkv, d, bs, dtype):
+    """Small batches with short contexts take the per-segment kernel (one block per (sequence, head
+    chunk), no workspace, no merge kernel): checked against the oracle, with an empty sequence and
+    ragged lengths up to 32 tiles, and against the split path (fixed chunks of one tile) on the same
+    inputs."""
+    import paged_kv_cache_457_b200 as pa
+    wl = W.custom(seed=500 + hq + hkv + d + bs, num_seqs=len(SEGMENT_LENS), num_q_heads=hq, num_kv_heads=hkv,
+                  head_dim=d, block_size=bs, lens=SEGMENT_LENS, dtype=dtype)
+    st = wl.steps[0]
+    assert pa.decode_workspace_size(st.num_seqs, hq, hkv, d, bs, st.max_context_len, 0) == 0, \
+        "expected the per-segment path (it needs no workspace)"
+    dev = DeviceState(wl)
+    dev.write(st)
+    seg = dev.decode(st, partition_tokens=0)
+    split = dev.decode(st, partition_tokens=16)
+    assert pa.device_status() == 0
+    _, _, ref = oracle_step(wl, wl.k_cache, wl.v_cache, st)
+    compare(seg, ref, dtype, what=f"segment path {hq}/{hkv} d{d} bs{bs} {dtype}")
+    compare(split, ref, dtype, what=f"split path {hq}/{hkv} d{d} bs{bs} {dtype}")
+    assert not np.any(seg[0])  # the empty sequence's rows are zero
+    assert np.array_equal(seg, dev.decode(st, partition_tokens=0)), "not deterministic"
+
+
+def test_small_batch_segment_path_one_full_wave():
+    """As many segments as the per-segment kernel takes in one wave of blocks (and one more, which
+    falls back to the split path), checked against the oracle on sampled sequences."""
+    import paged_kv_cache_457_b200 as pa
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rng = np.random.default_rng(7)
+    for extra in (0, 1):
+        S = None
+        # the largest batch of 8-head sequences the segment path accepts: S * 8 segments in one wave
+        for cand in range(sms * 4, 0, -1):
+            if pa.decode_workspace_size(cand, 8, 8, 64, 16, 200, 0) == 0:
+                S = cand
+                break
+        assert S is not None
+        S += extra
+        lens = [int(x) for x in rng.integers(1, 201, size=S)]
+        wl = W.custom(seed=600 + extra, num_seqs=S, num_q_heads=8, num_kv_heads=8, head_dim=64, block_size=16,
+                      lens=lens, dtype="fp16")
+        st = wl.steps[0]
+        assert (pa.decode_workspace_size(S, 8, 8, 64, 16, st.max_context_len, 0) == 0) == (extra == 0)
+        dev = DeviceState(wl)
+        dev.write(st)
+        out = dev.decode(st)
+        assert pa.device_status() == 0
+        seqs = np.sort(rng.choice(S, 12, replace=False))
+        _, _, ref = oracle_step(wl, wl.k_cache, wl.v_cache, st, seqs)
+        compare(out[seqs], ref, "fp16", what=f"{S} sequences")

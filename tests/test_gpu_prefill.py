@@ -124,8 +124,10 @@ def test_chunked_equals_whole_prompt():
 
 @pytest.mark.parametrize("name", sorted(W.PREFILL_NAMED))
 def test_full_size_sampled(name):
-    """The measured configurations at full size, in the launch the bench times; two sequences checked
-    row by row against the oracle, every row checked finite."""
+    """The measured configurations at full size, in the launch the bench times; the two shortest
+    sequences checked row by row against the oracle, and the first and last 64 rows of the longest
+    one (its lightest and heaviest rows: the last ones attend to the whole context); every row checked
+    finite."""
     require_gpu()
     case = W.PREFILL_NAMED[name]()
     got = run(case)
@@ -140,6 +142,20 @@ def test_full_size_sampled(name):
                                "query_start": np.array([0, qs[s + 1] - qs[s]], np.int32),
                                "context_lens": lens[s:s + 1], "block_tables": case.block_tables[s:s + 1]})
         compare(got[qs[s]:qs[s + 1]], expect(sub), case.dtype, what=f"{name} sequence {s}")
+    s = int(order[-1])
+    n, L = int(qs[s + 1] - qs[s]), int(lens[s])
+    k = min(64, n)
+    # the last k new tokens sit at positions L - k .. L - 1: a sub-case with k new tokens and the same context
+    last = W.PrefillCase(**{**case.__dict__, "q": case.q[qs[s + 1] - k:qs[s + 1]],
+                            "query_start": np.array([0, k], np.int32), "context_lens": lens[s:s + 1],
+                            "block_tables": case.block_tables[s:s + 1]})
+    compare(got[qs[s + 1] - k:qs[s + 1]], expect(last), case.dtype, what=f"{name} longest sequence, last rows")
+    # the first k new tokens sit at positions L - n .. L - n + k - 1: context L - n + k
+    first = W.PrefillCase(**{**case.__dict__, "q": case.q[qs[s]:qs[s] + k],
+                             "query_start": np.array([0, k], np.int32),
+                             "context_lens": np.array([L - n + k], np.int32),
+                             "block_tables": case.block_tables[s:s + 1]})
+    compare(got[qs[s]:qs[s] + k], expect(first), case.dtype, what=f"{name} longest sequence, first rows")
 
 
 def test_skewed_batch_one_long_prompt_among_decode_steps():
