@@ -6,6 +6,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads as W
 from gpu_util import DeviceState, compare, host_bits, oracle_step, require_gpu
 
@@ -162,3 +163,67 @@ def test_small_batch_segment_path_one_full_wave():
         seqs = np.sort(rng.choice(S, 12, replace=False))
         _, _, ref = oracle_step(wl, wl.k_cache, wl.v_cache, st, seqs)
         compare(out[seqs], ref, "fp16", what=f"{S} sequences")
+
+
+PAIR_SHAPES = [  # (hq, hkv, d, bs, dtype): tensor-core groups of 3 and 4 heads
+    (8, 2, 128, 16, "bf16"),
+    (8, 2, 64, 32, "fp16"),
+    (6, 2, 128, 32, "fp16"),
+    (12, 4, 64, 16, "bf16"),
+]
+# (L0, L1, blocks of the first sequence's table the second one names too: a prefix they share)
+PAIR_LENS = [(1040, 1040, 64), (300, 520, 10), (17, 900, 1), (900, 17, 1), (0, 50, 0), (70, 0, 0), (256, 256, 15),
+             (33, 2000, 2), (1, 1, 0), (640, 333, 0), (129, 129, 8), (47, 0, 0), (5000, 4000, 200)]
+
+
+def _paired_case(hq, hkv, d, bs, dtype, seed):
+    lens = [x for L0, L1, _ in PAIR_LENS for x in (L0, L1)] + [613]  # an odd batch: the last unit has one sequence
+    wl = W.custom(seed=seed, num_seqs=len(lens), num_q_heads=hq, num_kv_heads=hkv, head_dim=d, block_size=bs,
+                  lens=lens, dtype=dtype)
+    st = wl.steps[0]
+    tables = st.block_tables.copy()
+    for i, (L0, L1, blocks) in enumerate(PAIR_LENS):
+        # name the first sequence's leading blocks in the second one's table (a shared prefix); the new tokens
+        # written by the step stay in unshared blocks
+        share = min(blocks * 16 // bs, max(0, (min(L0, L1) - 1) // bs))
+        tables[2 * i + 1, :share] = tables[2 * i, :share]
+    return wl, st, tables
+
+
+@pytest.mark.parametrize("hq,hkv,d,bs,dtype", PAIR_SHAPES)
+@pytest.mark.parametrize("partition", [0, 16, 48])
+def test_shared_prefix_tables(hq, hkv, d, bs, dtype, partition):
+    """Consecutive sequences whose tables name the same leading blocks (shared prefixes of every length:
+    long, short, one block, none), an empty sequence on either side of such a pair, and an odd batch, on
+    the tensor-core path, against the oracle through the same tables, with the balanced split and with
+    chunks of 1 and 3 tiles (pieces cut inside the shared blocks and inside each sequence's own)."""
+    import paged_kv_cache_457_b200 as pa
+    wl, st, tables = _paired_case(hq, hkv, d, bs, dtype, seed=700 + hq + d + bs)
+    dev = DeviceState(wl)
+    dev.write(st)
+    out = dev.decode(st, partition_tokens=partition, tables=tables)
+    assert pa.device_status() == 0
+    kc, vc = oracle.write_kv(st.k_new, st.v_new, wl.k_cache, wl.v_cache, st.slot_mapping, wl.block_size)
+    ref = oracle.decode(st.q, kc, vc, tables, st.context_lens, wl.scale, wl.dtype)
+    compare(out, ref, dtype, what=f"shared prefixes {hq}/{hkv} d{d} bs{bs} {dtype} part {partition}")
+    for s, L in enumerate(st.context_lens):
+        if L == 0:
+            assert not np.any(out[s]), f"sequence {s} (empty) not zero"
+
+
+def test_shared_prefix_bad_block_zeroes_only_its_sequence():
+    """A table entry outside the pool in one of two sequences that share their first blocks zeroes that
+    sequence's rows only (and sets the status bit); its partner and the rest are exact."""
+    import paged_kv_cache_457_b200 as pa
+    wl, st, tables = _paired_case(8, 2, 128, 16, "bf16", seed=77)
+    tables[3, 25] = wl.num_blocks + 3  # sequence 3 (pair 1: 300 / 520 tokens, 10 shared blocks), its own part
+    dev = DeviceState(wl)
+    dev.write(st)
+    for part in (0, 48):
+        out = dev.decode(st, partition_tokens=part, tables=tables)
+        assert pa.device_status() == pa.DEV_ERR_BLOCK_ID
+        assert not np.any(out[3])
+        good = [s for s in range(st.num_seqs) if s != 3]
+        kc, vc = oracle.write_kv(st.k_new, st.v_new, wl.k_cache, wl.v_cache, st.slot_mapping, wl.block_size)
+        ref = oracle.decode(st.q[good], kc, vc, tables[good], st.context_lens[good], wl.scale, wl.dtype)
+        compare(out[good], ref, "bf16", what=f"the other sequences, part {part}")
