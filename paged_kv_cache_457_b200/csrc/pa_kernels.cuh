@@ -261,8 +261,14 @@ __device__ __forceinline__ ChunkPlan plan_chunks(const DecodeArgs &a, int tiles_
 // the workspace.  Block 0 installs (epoch << 32) in the counter word at the
 // start of the call (the epoch is non-zero and new for every call, and the
 // merge kernel leaves the word at 0), so a ticket drawn before the install is
-// recognised by its stale upper half and drawn again.  Tickets are requested
-// half a chunk ahead of need.
+// recognised by its stale upper half and drawn again.  A warp requests its
+// next ticket TICKET_AHEAD tiles before its current chunk runs out: late
+// enough that a slow warp does not reserve work a faster one could take (a
+// request half a chunk ahead pinned most of the queue to warps that were
+// still busy), early enough that the atomic's round trip is hidden behind
+// the tiles already in flight.
+constexpr int TICKET_AHEAD = 3;
+
 struct ChunkQueue {
   unsigned long long *word;
   unsigned epoch;
@@ -690,7 +696,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS) decode_split_kernel(co
       }
       advance_tile(prod.pos, pt, S, HC);
       --prod_left;
-      if (!requested && 2 * prod_left <= plan.length(prod_c)) {
+      if (!requested && prod_left <= TICKET_AHEAD) {
         queue.request(lane);
         requested = true;
       }

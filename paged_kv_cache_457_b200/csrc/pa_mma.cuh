@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(WARPS * 32, 12 / WARPS)
       }
       advance_tile(prod.pos, pt, S, HC);
       --prod_left;
-      if (!requested && 2 * prod_left <= plan.length(prod_c)) {
+      if (!requested && prod_left <= TICKET_AHEAD) {
         queue.request(lane);
         requested = true;
       }
