@@ -1,13 +1,18 @@
 // sm_100a kernels of the paged decode path.
 //
-//   write_kv_kernel          slot-mapped scatter of this step's new K/V rows
-//                            ("4. vLLM核心机制" section 4.3, layout of 4.2).
-//   decode_partition_kernel  attention of one query token per sequence over
-//                            the block-paged cache, reached through the
-//                            per-sequence block table ("4. vLLM核心机制" 4.2;
-//                            "vLLM：大型语言模型推理优化的革命性突破" 2.1).
-//   decode_reduce_kernel     merges the partial softmax states of sequences
-//                            split along the context into several units.
+//   write_kv_kernel        slot-mapped scatter of this step's new K/V rows
+//                          ("4. vLLM核心机制" section 4.3, layout of 4.2).
+//   decode_split_kernel    attention of one query token per sequence over the
+//                          block-paged cache, reached through the per-sequence
+//                          block table ("4. vLLM核心机制" 4.2; "vLLM：大型语言模型
+//                          推理优化的革命性突破" 2.1), on the CUDA cores, over a
+//                          balanced stream of 16-token tiles (the tensor-core
+//                          variant for query groups of 3 to 8 heads is in
+//                          pa_mma.cuh).
+//   decode_segment_kernel  the same attention for small batches: one block per
+//                          (sequence, head chunk), no workspace, no merge.
+//   decode_merge_kernel    merges the partial softmax states of the segments
+//                          that the split kernel cut across chunks.
 //
 // Cache layout: [num_blocks][num_kv_heads][block_size][head_dim], so the
 // 16 consecutive tokens of one (block, kv head) form one contiguous tile of
@@ -142,10 +147,11 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const WriteArgs a) {
 // valid, non-empty context owns nt(s) = ceil(L_s / 16) tiles per head chunk
 // (a head chunk = one kv head and up to 8 of its query heads).  All tiles are
 // laid in one stream, ordered by sequence, then head chunk, then tile, and the
-// stream is cut into equal chunks of consecutive tiles; the warps of the
-// split kernel take chunks round-robin.  With the default chunk length
-// (total tiles / warps) every warp gets the same number of tiles, whatever the
-// length mix.  The part of a chunk that falls in one (sequence, head chunk)
+// stream is cut into chunks of consecutive tiles (ChunkPlan): warp w of the
+// split kernel takes chunk w, and later chunks come from a queue (ChunkQueue),
+// so a warp that runs ahead takes more.  The boundaries depend only on the
+// lengths and the launch shape, never on timing, so the output is the same on
+// every run.  The part of a chunk that falls in one (sequence, head chunk)
 // is a piece: a piece that covers its whole segment writes the final output,
 // the others write a partial softmax state that the merge kernel combines.
 struct DecodeArgs {
