@@ -443,21 +443,25 @@ int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype,
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  // merge: one warp per query head on the tensor-core path (segments of 3 to 8 heads), one warp per segment
-  // (1 or 2 heads) on the CUDA-core path; eight warps per block.  Measured and dropped: merging in the
-  // tensor-core split kernel itself (the warp that stores a segment's last cut piece merges it, counted
-  // through per-segment arrival words): 179 against 167 us on the 32 query / 8 kv head batch and 62
-  // against 43 us on the shared-prefix step -- the merges then run one after another at the end of each
-  // warp's stream instead of in parallel across the merge grid.
-  const int hw = uses_mma(args.group) ? 1 : args.heads_per_unit;
+  // merge: on the tensor-core path (segments of 3 to 8 heads) one warp per two query heads of a segment (one
+  // per head for an odd group); on the CUDA-core path one warp per segment (1 or 2 heads); eight warps per
+  // block.  Two heads per warp halve the grid, so more of it is resident on the SMs that finish the split
+  // early instead of being scheduled after the split drains: 41.0 against 42.2 us on the shared-prefix step,
+  // 165.8 against 166.2 on the 32 query / 8 kv head batch; four heads per warp (158 registers) lost on the
+  // latter.  Measured and dropped: merging in the tensor-core split kernel itself (the warp that stores a
+  // segment's last cut piece merges it, counted through per-segment arrival words): 179 against 167 us on
+  // the 32 query / 8 kv head batch and 62 against 43 us on the shared-prefix step -- the merges then run one
+  // after another at the end of each warp's stream instead of in parallel across the merge grid.
+  const int hw = uses_mma(args.group) ? (args.heads_per_unit % 2 == 0 ? 2 : 1) : args.heads_per_unit;
   const long long warps = (long long)args.num_seqs * args.num_kv_heads * args.n_chunks * (args.heads_per_unit / hw);
   const dim3 mgrid((unsigned)((warps + 7) / 8)), mblock(256);
-  if (hw == 2)
-    e = launch_pdl(pa::decode_merge_kernel<E, D, 2, 8>, mgrid, mblock, 0, stream, args);
-  else if (uses_mma(args.group))
-    e = launch_pdl(pa::decode_merge_kernel<E, D, 1, 4>, mgrid, mblock, 0, stream, args);
+  if (!uses_mma(args.group))
+    e = hw == 2 ? launch_pdl(pa::decode_merge_kernel<E, D, 2, 8>, mgrid, mblock, 0, stream, args)
+                : launch_pdl(pa::decode_merge_kernel<E, D, 1, 16>, mgrid, mblock, 0, stream, args);
+  else if (hw == 2)
+    e = launch_pdl(pa::decode_merge_kernel<E, D, 2, 4>, mgrid, mblock, 0, stream, args);
   else
-    e = launch_pdl(pa::decode_merge_kernel<E, D, 1, 16>, mgrid, mblock, 0, stream, args);
+    e = launch_pdl(pa::decode_merge_kernel<E, D, 1, 4>, mgrid, mblock, 0, stream, args);
   if (e != cudaSuccess) return record(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return record(e);
