@@ -18,6 +18,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CASES = [
     "tests/test_gpu_parity.py::test_small_shapes",
     "tests/test_gpu_parity.py::test_small_batch_segment_path",
+    "tests/test_gpu_parity.py::test_many_short_sequences",
     "tests/test_gpu_parity.py::test_shared_prefix_tables",
     "tests/test_gpu_parity.py::test_shared_prefix_bad_block_zeroes_only_its_sequence",
     "tests/test_gpu_errors.py",

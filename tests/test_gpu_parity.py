@@ -103,6 +103,30 @@ def test_small_shapes(hq, hkv, d, bs, dtype, partition):
     compare(out, ref, dtype, what=f"{hq}/{hkv} d{d} bs{bs} {dtype} part {partition}")
 
 
+@pytest.mark.parametrize("hq,hkv,dtype", [(32, 8, "fp16"), (8, 8, "fp16")])
+def test_many_short_sequences(hq, hkv, dtype):
+    """3000 sequences of 1 to 32 tokens and six of 1000 (tensor-core and CUDA-core paths).  The split
+    kernels' tile prefix then takes 12 KB of shared memory per block (fewer blocks per SM), each thread
+    of its scan covers 24 sequences, most chunks hold many whole segments and the long ones are cut
+    across chunks: every output row against the oracle.  fp16 storage: contexts this short give outputs
+    up to about 4 in magnitude, where one bf16 ulp (2^-6) is already above the 1e-2 bound."""
+    rng = np.random.default_rng(77)
+    lens = rng.integers(1, 33, size=3000)
+    lens[::500] = 1000
+    wl = W.custom(seed=78, num_seqs=len(lens), num_q_heads=hq, num_kv_heads=hkv, head_dim=128, block_size=16,
+                  lens=lens, dtype=dtype)
+    st = wl.steps[0]
+    dev = DeviceState(wl)
+    dev.write(st)
+    out = dev.decode(st)
+    import paged_kv_cache_457_b200 as pa
+    assert pa.device_status() == 0
+    _, _, ref = oracle_step(wl, wl.k_cache, wl.v_cache, st)
+    compare(out, ref, dtype, what=f"3006 seqs {hq}/{hkv} {dtype}")
+    del dev
+    _free()
+
+
 SEGMENT_SHAPES = [  # (hq, hkv, d, bs, dtype): CUDA-core groups of 1 and 2 heads
     (8, 8, 64, 16, "fp16"),
     (8, 8, 128, 32, "bf16"),
