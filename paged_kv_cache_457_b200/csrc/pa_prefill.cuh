@@ -83,6 +83,17 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for the share of the softmax's exponentials taken off the SFU (x <= RESCALE_SLACK;
+// x below -126, -inf included, gives 0).  2^x = 2^n * 2^f with n = round(x) -- adding 1.5 * 2^23 leaves n in
+// the low mantissa bits -- and f = x - n in [-1/2, 1/2]; 2^f by a cubic fitted to 2^f on [-1/2, 1/2] (least
+// squares at Chebyshev nodes, reweighted toward equal relative error: at most 7.5e-5, below the 2-byte rounding
+// of P that follows); n is then added to the exponent field.
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 // c + lo + hi of two packed 2-byte values, widened exactly by the mixed-precision fma (times 1.0):
 // the row sum adds the rounded P values that the PV product uses, so the weights sum to one.
 template <class E>
@@ -511,10 +522,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           for (int c = 0; c < PF_BN; ++c)
             if (key0 + c > vis) sv[c] = -INFINITY;
         }
-        // row max of the raw scores in four chains (scale_log2 > 0 keeps the order)
+        // row max of the raw scores in four chains, two scores per three-input max (scale_log2 > 0 keeps the order)
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < PF_BN; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], sv[c]);
+        for (int c = 0; c < PF_BN; c += 8)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) mx4[u] = fmax3(mx4[u], sv[c + u], sv[c + 4 + u]);
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
         const float m_new = fmaxf(m, mx);
         const bool need = m_new > m + RESCALE_SLACK;
@@ -532,8 +545,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             // masked scores are -inf: 2^-inf = 0
-            const float p0 = ex2(fmaf(sv[c * 32 + 2 * i], a.scale_log2, -m));
-            const float p1 = ex2(fmaf(sv[c * 32 + 2 * i + 1], a.scale_log2, -m));
+            // scale and shift two scores in one packed fma
+            const float2 x = __ffma2_rn(make_float2(sv[c * 32 + 2 * i], sv[c * 32 + 2 * i + 1]),
+                                        make_float2(a.scale_log2, a.scale_log2), make_float2(-m, -m));
+            const float p0 = ex2(x.x);
+            const float p1 = ex2(x.y);
             pk[i] = E::narrow2(p0, p1);
             sum4[i & 3] = add_packed<E>(pk[i], sum4[i & 3]);
           }
