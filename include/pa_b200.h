@@ -72,6 +72,8 @@ extern "C" {
 #define PA_DEV_ERR_SLOT 0x8u        /* a slot_mapping entry >= num_blocks * block_size */
 #define PA_DEV_ERR_TIMEOUT 0x10u    /* a bounded wait on a bulk copy ran out */
 #define PA_DEV_ERR_INTERNAL 0x20u   /* debug builds only: an internal index check failed; that access was skipped */
+#define PA_DEV_ERR_PLAN 0x40u       /* a cascade plan disagrees with the call: a group member's table differs on the
+                                       shared prefix or its context ends inside it, or a plan index is out of range */
 
 /* ---- build flags (pa_build_flags) ---- */
 #define PA_BUILD_DEBUG 0x1u /* built with PA_DEBUG: every derived index is checked on the device before use */
@@ -322,6 +324,95 @@ int pa_read_bandwidth_probe(const void *src, int64_t bytes, uint32_t *sink, void
  * build's.  It stands in for a memory checker on small cases.
  */
 uint32_t pa_build_flags(void);
+
+/* ---- cascade decode: shared-prefix groups read once ("4. vLLM核心机制" section 4.2) ----
+ *
+ * When several sequences' tables name the same leading blocks (one prompt
+ * sampled several times, a shared system prompt: the pages' copy-free prefix
+ * sharing), pa_decode reads those blocks once per sequence.  The cascade
+ * calls compute the same attention with every shared tile fetched once per
+ * group: the host finds the groups (pa_find_prefix_groups) and builds a plan
+ * (pa_cascade_plan), the caller copies the plan to the device with the
+ * step's other inputs, and pa_decode_cascade runs it.  The plan depends on
+ * the groups, the head counts, block_size and max_context_len only, not on
+ * the exact lengths, so a plan serves every step until a group changes.
+ */
+typedef struct pa_cascade_info {
+  int32_t num_seqs, num_q_heads, num_kv_heads, block_size, max_context_len;
+  int32_t num_jobs;      /* jobs: num_prefix_jobs prefix jobs first, then the suffix jobs */
+  int32_t num_prefix_jobs;
+  int32_t num_members;   /* entries of the plan's member list */
+  int32_t num_pieces;    /* partial states merged per (sequence, head) in total over the sequences */
+  int32_t rows_per_head; /* partial rows of the workspace per kv head */
+  int64_t plan_ints;     /* int32 entries of the plan */
+} pa_cascade_info;
+
+/*
+ * pa_find_prefix_groups -- host-side grouping of a batch by shared leading
+ * blocks.  All pointers are HOST memory.  block_tables int32
+ * [num_seqs][block_table_stride], context_lens int32 [num_seqs].  Sequences
+ * whose first table entries agree form a candidate group (only full blocks,
+ * j < context_len / block_size, count); its prefix is the longest run of
+ * leading entries every member shares.  A group is reported when it has at
+ * least two members and prefix >= max(1, min_prefix_blocks).  Output (caller
+ * arrays of num_seqs + 1, num_seqs, num_seqs int32): group g's members are
+ * group_members[group_offsets[g] .. group_offsets[g+1]) in increasing order,
+ * sharing group_prefix_blocks[g] blocks; groups are ordered by first member;
+ * *num_groups is their count.  Sequences in no group are not listed.
+ * Contexts outside [0, block_table_stride * block_size] -> PA_ERR_SHAPE.
+ */
+int pa_find_prefix_groups(const int32_t *block_tables, const int32_t *context_lens, int32_t num_seqs,
+                          int32_t block_table_stride, int32_t block_size, int32_t min_prefix_blocks,
+                          int32_t *group_offsets, int32_t *group_members, int32_t *group_prefix_blocks,
+                          int32_t *num_groups);
+
+/*
+ * pa_cascade_plan -- host-side work plan of pa_decode_cascade.  All pointers
+ * are HOST memory.  Groups as pa_find_prefix_groups reports them (any
+ * sequence at most once; sequences in no group, and groups with a zero
+ * prefix, attend through their own tables only); every member of group g
+ * must hold at least group_prefix_blocks[g] * block_size tokens, and
+ * group_prefix_blocks[g] * block_size <= max_context_len.  num_q_heads /
+ * num_kv_heads must be at most 8 (PA_ERR_UNSUPPORTED otherwise).
+ * chunk_tokens: tokens per job along the context, 0 = 256, else a positive
+ * multiple of 16 (PA_ERR_PARTITION).  Fills *info; writes the plan
+ * (info->plan_ints int32) to `plan` unless it is NULL (a size query).
+ * plan_capacity (entries) smaller than needed -> PA_ERR_WORKSPACE, with
+ * *info filled.
+ * Jobs: per group, per column set of up to 4 * (8 / G) members, per chunk
+ * of the shared tiles; per sequence, per chunk of the tiles from its
+ * prefix to ceil(max_context_len / 16).
+ */
+int pa_cascade_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t block_size,
+                    int32_t max_context_len, int32_t chunk_tokens, int32_t num_groups, const int32_t *group_offsets,
+                    const int32_t *group_members, const int32_t *group_prefix_blocks, int32_t *plan,
+                    int64_t plan_capacity, pa_cascade_info *info);
+
+/* pa_cascade_workspace_size -- device workspace bytes pa_decode_cascade needs for this plan (0 on bad input). */
+size_t pa_cascade_workspace_size(const pa_cascade_info *info, int32_t head_dim);
+
+/*
+ * pa_decode_cascade -- the attention of pa_decode (same definition, same
+ * fp32 arithmetic, rounded to nearest even), computed by the plan's jobs:
+ * each job streams 16-token tiles of one table row once and applies them to
+ * all of its members' query heads, leaving partial softmax states in the
+ * workspace; a second kernel merges every (sequence, head)'s pieces in plan
+ * order (deterministic).  Sizes (num_seqs, heads, block_size,
+ * max_context_len) come from *info (host); `plan` is the plan in DEVICE
+ * memory, unchanged until the call has run.  Other arguments as pa_decode.
+ * Device-side errors: a context outside [0, min(block_table_stride *
+ * block_size, max_context_len)] -> zero row and PA_DEV_ERR_CONTEXT(_HINT);
+ * a member whose table differs from its group's first member on the shared
+ * blocks, or whose context ends inside them, or a plan index out of range
+ * -> PA_DEV_ERR_PLAN and zero rows for the sequences concerned; table
+ * entries outside the pool -> PA_DEV_ERR_BLOCK_ID and zero rows.
+ * info->num_seqs == 0 launches nothing.
+ */
+int pa_decode_cascade(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                      const int32_t *context_lens, float scale, void *out, int32_t head_dim, int64_t num_blocks,
+                      int32_t block_table_stride, int64_t q_seq_stride, int64_t out_seq_stride, int32_t dtype,
+                      const int32_t *plan, const pa_cascade_info *info, void *workspace, size_t workspace_bytes,
+                      void *stream);
 
 /* pa_version -- library ABI version (major * 10000 + minor * 100 + patch). */
 int32_t pa_version(void);

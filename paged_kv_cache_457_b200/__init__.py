@@ -9,6 +9,9 @@ CPU fallback: if the library is missing or no GPU is present the calls raise.
 * :func:`decode`   -- single-token attention over the block-paged cache through
   per-sequence block tables ("4. vLLM核心机制", section 4.2;
   "vLLM：大型语言模型推理优化的革命性突破", section 2.1).
+* :func:`decode_cascade` -- the same attention for batches whose tables share
+  leading blocks, each shared tile read once per group ("4. vLLM核心机制",
+  section 4.2), with :func:`find_prefix_groups` and :func:`cascade_plan` on the host.
 
 Caches are ``[num_blocks, num_kv_heads, block_size, head_dim]`` float16 or
 bfloat16 tensors; ``block_tables`` int32 ``[S, max_blocks]``; ``context_lens``
@@ -29,6 +32,8 @@ __all__ = [
     "DEV_ERR_BLOCK_ID", "DEV_ERR_CONTEXT", "DEV_ERR_CONTEXT_HINT", "DEV_ERR_SLOT", "DEV_ERR_TIMEOUT",
     "DEV_ERR_INTERNAL", "BUILD_DEBUG", "build_flags",
     "BlockManager", "BlockManagerError", "DecodeStepPlan", "PrefillStepPlan",
+    "DEV_ERR_PLAN", "find_prefix_groups", "cascade_plan", "cascade_workspace_size", "decode_cascade", "PrefixGroups",
+    "CascadePlan",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,6 +47,7 @@ DEV_ERR_CONTEXT_HINT = 0x4
 DEV_ERR_SLOT = 0x8
 DEV_ERR_TIMEOUT = 0x10
 DEV_ERR_INTERNAL = 0x20
+DEV_ERR_PLAN = 0x40
 BUILD_DEBUG = 0x1
 
 _DTYPES = {torch.float16: 1, torch.bfloat16: 2}
@@ -54,6 +60,7 @@ EXPORTED_SYMBOLS = (
     "pa_bm_ref_count", "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_num_tokens",
     "pa_bm_is_swapped", "pa_bm_block_table", "pa_bm_slots", "pa_bm_append_slot", "pa_bm_build_decode_step", "pa_bm_build_prefill_step", "pa_bm_step_needs",
     "pa_bm_swap_out", "pa_bm_swap_in", "pa_prefill", "pa_read_bandwidth_probe", "pa_build_flags",
+    "pa_find_prefix_groups", "pa_cascade_plan", "pa_cascade_workspace_size", "pa_decode_cascade",
 )
 
 
@@ -113,7 +120,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_version.restype = i32
         lib.pa_version.argtypes = []
         from .block_manager import bind as _bind_block_manager
+        from .cascade import bind as _bind_cascade
         _bind_block_manager(lib)
+        _bind_cascade(lib)
         if path is None:
             _lib = lib
         return lib
@@ -347,3 +356,5 @@ def debug_wait_timeout(limit_ns: int = 10_000_000) -> None:
 
 
 from .block_manager import BlockManager, BlockManagerError, DecodeStepPlan, PrefillStepPlan  # noqa: E402
+from .cascade import (CascadePlan, PrefixGroups, cascade_plan, cascade_workspace_size,  # noqa: E402
+                      decode_cascade, find_prefix_groups)

@@ -19,8 +19,10 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpa_b200.so")
 # the same sources with PA_DEBUG: every index the kernels derive is checked on the device before use
 DEBUG_LIB = os.path.join(PKG, "libpa_b200_debug.so")
-SOURCES = [os.path.join(CSRC, "pa_api.cu"), os.path.join(CSRC, "block_manager.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_mma.cuh", "pa_ptx.cuh", "pa_copy.cuh", "pa_prefill.cuh", "pa_tcgen05.cuh", "pa_stream.cuh")] + [
+SOURCES = [os.path.join(CSRC, "pa_api.cu"), os.path.join(CSRC, "block_manager.cpp"),
+           os.path.join(CSRC, "cascade_plan.cpp")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("pa_kernels.cuh", "pa_mma.cuh", "pa_ptx.cuh", "pa_copy.cuh", "pa_prefill.cuh", "pa_tcgen05.cuh", "pa_stream.cuh", "pa_cascade.cuh",
+                                                   "pa_plan_layout.h")] + [
     os.path.join(INCLUDE, h) for h in ("pa_b200.h", "pa_block_manager.h")]
 
 

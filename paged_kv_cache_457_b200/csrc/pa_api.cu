@@ -15,6 +15,7 @@
 #include <cudaTypedefs.h>
 
 #include "pa_b200.h"
+#include "pa_cascade.cuh"
 #include "pa_copy.cuh"
 #include "pa_kernels.cuh"
 #include "pa_prefill.cuh"
@@ -469,6 +470,52 @@ int launch_decode_d(const pa::DecodeArgs &args, const LaunchPlan &lp, int dtype,
   return PA_OK;
 }
 
+// Workspace of a cascade plan: per kv head, rows_per_head softmax states (m, l) and partial rows acc[D].
+size_t cascade_ml_bytes(const pa_cascade_info &in) {
+  return ((size_t)in.num_kv_heads * (size_t)in.rows_per_head * sizeof(float2) + 255) / 256 * 256;
+}
+size_t cascade_ws_bytes(const pa_cascade_info &in, int head_dim) {
+  return std::max<size_t>(256, cascade_ml_bytes(in) + (size_t)in.num_kv_heads * (size_t)in.rows_per_head *
+                                                          (size_t)head_dim * sizeof(float));
+}
+
+static_assert(pa::CASCADE_CONSUMERS == kWarps, "blocks_per_sm sizes the cascade blocks with kWarps warps");
+
+template <class E, int D>
+int launch_cascade_d(const pa::CascadeArgs &a, const void *k_cache, const void *v_cache, int dtype,
+                     cudaStream_t stream) {
+  if (a.num_jobs > 0) {
+    const long long rows = a.num_blocks * a.num_kv_heads * a.block_size;
+    if (rows > 0x7fffffffLL) return PA_ERR_SHAPE;  // TMA coordinates are signed 32-bit
+    CUtensorMap mk, mv;
+    int rc = cache_tensor_map(k_cache, rows, D, dtype, true, &mk);
+    if (rc != PA_OK) return rc;
+    rc = cache_tensor_map(v_cache, rows, D, dtype, true, &mv);
+    if (rc != PA_OK) return rc;
+    // one block per prefix job, one per CASCADE_CONSUMERS suffix jobs
+    const long long blocks = a.num_prefix_jobs + ((long long)(a.num_jobs - a.num_prefix_jobs) + pa::CASCADE_CONSUMERS - 1) /
+                                                     pa::CASCADE_CONSUMERS;
+    int per_sm = 0;
+    rc = blocks_per_sm(reinterpret_cast<const void *>(pa::cascade_partial_kernel<E, D>), pa::CascadeSmem<D>::bytes(),
+                       &per_sm);  // also allows the kernel its shared memory above the default 48 KB
+    if (rc != PA_OK) return rc;
+    cudaError_t e = launch_pdl(pa::cascade_partial_kernel<E, D>, dim3((unsigned)blocks, (unsigned)a.num_kv_heads),
+                               dim3(pa::CASCADE_CONSUMERS * 32), pa::CascadeSmem<D>::bytes(), stream, mk, mv, a);
+    if (e != cudaSuccess) return record(e);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return record(e);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  const long long warps = (long long)a.num_seqs * a.num_q_heads;
+  cudaError_t e = launch_pdl(pa::cascade_combine_kernel<E, D>, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0,
+                             stream, a);
+  if (e != cudaSuccess) return record(e);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return record(e);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return PA_OK;
+}
+
 // Fixed scratch behind pa_decode_static_workspace, for callers that cannot
 // allocate.  In host code this name is only a stand-in for the device
 // variable: the kernels are given the address cudaGetSymbolAddress returns.
@@ -621,6 +668,73 @@ int pa_decode(const void *q, const void *k_cache, const void *v_cache, const int
   if (head_dim == 128)
     return bf16 ? launch_decode_d<pa::BF16, 128>(a, lp, dtype, st) : launch_decode_d<pa::F16, 128>(a, lp, dtype, st);
   return bf16 ? launch_decode_d<pa::BF16, 64>(a, lp, dtype, st) : launch_decode_d<pa::F16, 64>(a, lp, dtype, st);
+}
+
+size_t pa_cascade_workspace_size(const pa_cascade_info *info, int32_t head_dim) {
+  if (!info || (head_dim != 64 && head_dim != 128) || info->num_kv_heads <= 0 || info->rows_per_head < 0) return 0;
+  return cascade_ws_bytes(*info, head_dim);
+}
+
+int pa_decode_cascade(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                      const int32_t *context_lens, float scale, void *out, int32_t head_dim, int64_t num_blocks,
+                      int32_t block_table_stride, int64_t q_seq_stride, int64_t out_seq_stride, int32_t dtype,
+                      const int32_t *plan, const pa_cascade_info *info, void *workspace, size_t workspace_bytes,
+                      void *stream) {
+  if (!info) return PA_ERR_NULL;
+  const pa_cascade_info in = *info;
+  int rc = check_decode_shape(in.num_seqs, in.num_q_heads, in.num_kv_heads, head_dim, in.block_size,
+                              in.max_context_len);
+  if (rc != PA_OK) return rc;
+  if (in.num_q_heads / in.num_kv_heads > 8) return PA_ERR_UNSUPPORTED;
+  if (dtype != PA_FLOAT16 && dtype != PA_BFLOAT16) return PA_ERR_DTYPE;
+  if (num_blocks <= 0 || block_table_stride <= 0) return PA_ERR_SHAPE;
+  const int64_t row = (int64_t)in.num_q_heads * head_dim;
+  if (q_seq_stride < row || out_seq_stride < row) return PA_ERR_SHAPE;
+  if (in.num_jobs < 0 || in.num_prefix_jobs < 0 || in.num_prefix_jobs > in.num_jobs || in.num_members < 0 || in.num_pieces < 0 || in.rows_per_head < 0 ||
+      in.plan_ints != (int64_t)in.num_jobs * pa::CJ_INTS + in.num_members + in.num_seqs + 1 + in.num_pieces)
+    return PA_ERR_SHAPE;
+  if (in.num_seqs == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out || !plan) return PA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || (q_seq_stride % 8) ||
+      (out_seq_stride % 8))
+    return PA_ERR_ALIGN;
+  if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if (!workspace || workspace_bytes < cascade_ws_bytes(in, head_dim) || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+
+  pa::CascadeArgs a;
+  a.q = static_cast<const uint16_t *>(q);
+  a.out = static_cast<uint16_t *>(out);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.jobs = plan;
+  a.members = plan + (int64_t)in.num_jobs * pa::CJ_INTS;
+  a.piece_offsets = a.members + in.num_members;
+  a.piece_rows = a.piece_offsets + in.num_seqs + 1;
+  a.ws_ml = reinterpret_cast<float2 *>(workspace);
+  a.ws_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) + cascade_ml_bytes(in));
+  a.q_seq_stride = q_seq_stride;
+  a.out_seq_stride = out_seq_stride;
+  a.num_blocks = num_blocks;
+  a.wait_limit_ns = kWaitLimitNs;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);  // log2(e)
+  a.num_seqs = in.num_seqs;
+  a.num_q_heads = in.num_q_heads;
+  a.num_kv_heads = in.num_kv_heads;
+  a.block_size = in.block_size;
+  a.table_stride = block_table_stride;
+  a.max_context_len = in.max_context_len;
+  a.group = in.num_q_heads / in.num_kv_heads;
+  a.num_jobs = in.num_jobs;
+  a.num_prefix_jobs = in.num_prefix_jobs;
+  a.num_members = in.num_members;
+  a.num_pieces = in.num_pieces;
+  a.rows_per_head = in.rows_per_head;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PA_BFLOAT16)
+    return head_dim == 128 ? launch_cascade_d<pa::BF16, 128>(a, k_cache, v_cache, dtype, st)
+                           : launch_cascade_d<pa::BF16, 64>(a, k_cache, v_cache, dtype, st);
+  return head_dim == 128 ? launch_cascade_d<pa::F16, 128>(a, k_cache, v_cache, dtype, st)
+                         : launch_cascade_d<pa::F16, 64>(a, k_cache, v_cache, dtype, st);
 }
 
 int pa_get_device_status(uint32_t *status_out, int32_t clear, void *stream) {
