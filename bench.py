@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--prefill-workload", default="llama2_7b_prefill", choices=sorted(W.PREFILL_NAMED))
     ap.add_argument("--pairs", type=int, default=None, help="block pairs per step (block operations)")
     ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--cascade", default="auto", choices=["auto", "on", "off"],
+                    help="decode through pa_decode_cascade (prefix groups found on the host from the step's tables); "
+                         "auto: when the batch has groups and no fixed partition is asked for")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0,
@@ -742,14 +745,29 @@ def main():
                                         mcl, part)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
 
+    # Shared leading blocks: the host finds the groups from the step's tables (as a scheduler would) and the
+    # cascade path reads each group's shared tiles once.
+    groups = pa.find_prefix_groups(st.block_tables, st.context_lens, wl.block_size)
+    use_cascade = args.cascade == "on" or (args.cascade == "auto" and groups.num_groups > 0 and part == 0)
+    if use_cascade:
+        plan = pa.cascade_plan(st.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.block_size, mcl, groups)
+        plan_dev = plan.to(device)
+        cws = torch.empty(max(pa.cascade_workspace_size(plan, wl.head_dim), 16), dtype=torch.uint8, device=device)
+
+    def decode_into(q_, tables_, lens_, out_, plan_dev_=None):
+        if use_cascade:
+            pa.decode_cascade(q_, k_cache, v_cache, tables_, lens_, wl.scale, plan,
+                              plan_dev if plan_dev_ is None else plan_dev_, out=out_, workspace=cws)
+        else:
+            pa.decode(q_, k_cache, v_cache, tables_, lens_, wl.scale, max_context_len=mcl, out=out_,
+                      partition_tokens=part, workspace=ws)
+
     def step():
         pa.write_kv(k_new, v_new, k_cache, v_cache, slots)
-        pa.decode(q, k_cache, v_cache, tables, lens, wl.scale, max_context_len=mcl, out=out,
-                  partition_tokens=part, workspace=ws)
+        decode_into(q, tables, lens, out)
 
     def decode_only():
-        pa.decode(q, k_cache, v_cache, tables, lens, wl.scale, max_context_len=mcl, out=out,
-                  partition_tokens=part, workspace=ws)
+        decode_into(q, tables, lens, out)
 
     kv_b, alg_b = step_bytes(wl, st)
     uniq_kv = W.unique_kv_bytes(st, wl.num_kv_heads, wl.head_dim, wl.block_size)
@@ -883,6 +901,8 @@ def main():
         # as a serving loop would: one transfer per step instead of one per tensor keeps the host ahead.
         parts = [("q", st.q, q), ("k", st.k_new, k_new), ("v", st.v_new, v_new), ("slots", st.slot_mapping, slots),
                  ("tables", st.block_tables, tables), ("lens", st.context_lens, lens)]
+        if use_cascade:
+            parts.append(("plan", plan.plan, plan_dev))
         offsets, total = {}, 0
         for n, arr, _ in parts:
             offsets[n] = total
@@ -927,8 +947,7 @@ def main():
             compute.wait_event(ready[b])
             compute.wait_event(drained[b])
             pa.write_kv(buf["k"], buf["v"], k_cache, v_cache, buf["slots"])
-            pa.decode(buf["q"], k_cache, v_cache, buf["tables"], buf["lens"], wl.scale, max_context_len=mcl,
-                      out=buf["out"], partition_tokens=part, workspace=ws)
+            decode_into(buf["q"], buf["tables"], buf["lens"], buf["out"], buf.get("plan"))
             computed[b].record(compute)
             with torch.cuda.stream(d2h_stream):
                 d2h_stream.wait_event(computed[b])
@@ -956,7 +975,9 @@ def main():
                "ms_per_step": round(e2e_ms / args.steps, 4),
                "how": "each step's inputs copied from one pinned host buffer (one copy per step) and its output "
                       "read back, on two copy streams, double-buffered so that they overlap the previous step's "
-                      "kernels"}
+                      "kernels" + ("; the cascade plan is among the copied inputs (built on the host once for the "
+                                   "batch's groups, as a scheduler rebuilds it only when a group changes)"
+                                   if use_cascade else "")}
 
     elapsed_ms, dec_ms, read_peak_neg = max_over_ranks([elapsed_ms, dec_ms, -read_peak], device)
     read_peak = -read_peak_neg  # the slowest rank's probe
@@ -971,7 +992,8 @@ def main():
         value_distinct = job_rate_gbs(uniq_kv, world, args.steps, elapsed_ms)
         peak, peak_kind = measured_peak()
         achieved = alg_unique / (dec_ms / 1e3) / 1e9
-        traffic, traffic_note = recorded_traffic(wl.name)
+        traffic, traffic_note = recorded_traffic(wl.name) if not use_cascade else (
+            None, "no ncu capture of the cascade kernels")
         shared = uniq_kv != kv_b
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -990,11 +1012,17 @@ def main():
                        "parallelism": f"dp{world} (independent batches per GPU)",
                        "timing": ("per-step CUDA events, L2 flushed before each step" if flush else
                                   "one CUDA event pair around all steps, back to back")
-                       + ("; each step a replay of a CUDA graph of pa_write_kv + pa_decode" if not args.no_graph
+                       + ((f"; each step a replay of a CUDA graph of pa_write_kv + "
+                           f"{'pa_decode_cascade' if use_cascade else 'pa_decode'}") if not args.no_graph
                           else "; direct library calls"),
+                       "path": (f"pa_decode_cascade: {groups.num_groups} prefix groups found on the host "
+                                f"(sizes {sorted(set(np.diff(groups.offsets).tolist()))}, shared blocks "
+                                f"{sorted(set(groups.prefix_blocks.tolist()))}), each shared tile read once per group"
+                                if use_cascade else "pa_decode"),
                        "l2": l2_note(flush, alg_unique, l2_bytes, flush_bytes)},
             "step_timing": summarize_ms(step_times) if step_times else None,
-            "roofline": {"bound": "hbm", "kernel": "pa_decode (split + merge kernels)",
+            "roofline": {"bound": "hbm", "kernel": ("pa_decode_cascade (partial + combine kernels)" if use_cascade
+                                                    else "pa_decode (split + merge kernels)"),
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic, "traffic_note": traffic_note,
                          "algorithmic_bytes": alg_unique,

@@ -98,17 +98,20 @@ int pa_cascade_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
     }
 
   const int32_t max_tiles = (max_context_len + pa::CASCADE_TILE - 1) / pa::CASCADE_TILE;
-  const int32_t per_job = pa::CASCADE_CONSUMERS * (8 / G);  // members whose heads fit one block's columns
+  // a prefix job's members fill up to CASCADE_CONSUMERS row tiles of 16 (member, head) rows; a job with fewer
+  // row tiles deals its tiles to `split` sets of warps so that every warp of the block works
+  const int32_t per_tile = 16 / G;
+  const int32_t per_job = pa::CASCADE_CONSUMERS * per_tile;
   std::vector<int32_t> jobs, members;
   std::vector<std::vector<int32_t>> pieces(num_seqs);  // partial rows of each sequence, in merge order
   int64_t rows = 0;
-  auto add_job = [&](int32_t seq, int32_t t0, int32_t t1, int32_t mfirst, int32_t nm, int32_t kind) {
-    const int32_t job[pa::CJ_INTS] = {seq, t0, t1, mfirst, nm, (int32_t)rows, kind, 0};
+  auto add_job = [&](int32_t seq, int32_t t0, int32_t t1, int32_t mfirst, int32_t nm, int32_t kind, int32_t split) {
+    const int32_t job[pa::CJ_INTS] = {seq, t0, t1, mfirst, nm, (int32_t)rows, kind, split};
     static_assert(pa::CJ_SEQ == 0 && pa::CJ_T0 == 1 && pa::CJ_T1 == 2 && pa::CJ_MEMBERS == 3 && pa::CJ_NM == 4 &&
-                      pa::CJ_ROW == 5 && pa::CJ_KIND == 6 && pa::CJ_INTS == 8,
+                      pa::CJ_ROW == 5 && pa::CJ_KIND == 6 && pa::CJ_SPLIT == 7 && pa::CJ_INTS == 8,
                   "job fields in the order written here");
     jobs.insert(jobs.end(), job, job + pa::CJ_INTS);
-    rows += (int64_t)nm * G;
+    rows += (int64_t)nm * G * split;
   };
   // prefix jobs first (the long ones start early): per group, per column set, per chunk of the shared tiles
   for (int32_t g = 0; g < num_groups; ++g) {
@@ -120,10 +123,14 @@ int pa_cascade_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
     const int32_t lead = group_members[group_offsets[g]];
     for (int32_t c0 = 0; c0 < n; c0 += per_job) {
       const int32_t nm = std::min(per_job, n - c0);
+      const int32_t n_rt = (nm + per_tile - 1) / per_tile;
+      const int32_t split = n_rt == 1 ? 4 : n_rt == 2 ? 2 : 1;
       for (int32_t t0 = 0; t0 < PT; t0 += CH) {
         const int64_t row = rows;
-        add_job(lead, t0, std::min(PT, t0 + CH), mlist + c0, nm, pa::CJ_PREFIX);
-        for (int32_t i = 0; i < nm; ++i) pieces[members[mlist + c0 + i]].push_back((int32_t)(row + (int64_t)i * G));
+        add_job(lead, t0, std::min(PT, t0 + CH), mlist + c0, nm, pa::CJ_PREFIX, split);
+        for (int32_t sp = 0; sp < split; ++sp)
+          for (int32_t i = 0; i < nm; ++i)
+            pieces[members[mlist + c0 + i]].push_back((int32_t)(row + ((int64_t)sp * nm + i) * G));
       }
     }
   }
@@ -134,7 +141,7 @@ int pa_cascade_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
   for (int32_t s = 0; s < num_seqs; ++s)
     for (int32_t t0 = prefix_tiles[s]; t0 < max_tiles; t0 += CH) {
       pieces[s].push_back((int32_t)rows);
-      add_job(s, t0, std::min(max_tiles, t0 + CH), self + s, 1, pa::CJ_SUFFIX);
+      add_job(s, t0, std::min(max_tiles, t0 + CH), self + s, 1, pa::CJ_SUFFIX, 1);
     }
   if (rows > INT32_MAX / 2) return PA_ERR_SHAPE;
 

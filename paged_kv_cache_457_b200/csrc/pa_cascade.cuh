@@ -29,6 +29,9 @@ namespace pa {
 static_assert(CASCADE_TILE == TILE, "one plan tile is one ring tile");
 constexpr int CASCADE_SLOTS = 8;  // ring slots per block: all shared by a prefix job, two per warp for suffix jobs
 constexpr int CASCADE_WARP_SLOTS = CASCADE_SLOTS / CASCADE_CONSUMERS;
+#ifndef CASCADE_MIN_BLOCKS
+#define CASCADE_MIN_BLOCKS 3
+#endif
 
 struct CascadeArgs {
   const uint16_t *q;
@@ -75,7 +78,9 @@ struct RowWindow {
 };
 
 // Lane 0: K and V of tile t of (block phys, kv head h), one 3-D TMA box each, into `dst`, completing on `bar`;
-// an entry outside the pool flags the slot instead and completes the barrier without data.
+// an entry outside the pool flags the slot instead and completes the barrier without data.  The caller has
+// fenced the generic-proxy reads of the slot's previous contents against the copy (fence_proxy_async_smem, once
+// for any number of copies issued after it).
 template <int D>
 __device__ __forceinline__ void cascade_issue(const CascadeArgs &a, const CUtensorMap *mk, const CUtensorMap *mv,
                                               int phys, int t, int h, unsigned char *dst, uint64_t *bar, int *bad) {
@@ -84,7 +89,6 @@ __device__ __forceinline__ void cascade_issue(const CascadeArgs &a, const CUtens
   *bad = ok ? 0 : 1;
   if (ok) {
     const int row = (int)(((long long)phys * a.num_kv_heads + h) * a.block_size + (t * TILE) % a.block_size);
-    fence_proxy_async_smem();  // the slot's previous contents were read through the generic proxy
     mbar_arrive_expect_tx(bar, 2 * TILE_BYTES);
     tc::tma_load_3d(dst, mk, 0, row, 0, bar);
     tc::tma_load_3d(dst + TILE_BYTES, mv, 0, row, 0, bar);
@@ -219,18 +223,159 @@ struct ColumnTile {
   }
 };
 
-// One job of the plan, read and checked (the plan lives in the caller's memory).
+// One warp's 16 query rows (row r: member r / G of the warp's row tile, head r % G) against a 16-token tile, with
+// the queries as the mma's M dimension (prefix jobs, where many rows share each tile):
+//   S[16 rows x 16 tokens]  = Q[16 x d] . K^T[d x 16]        (two 8-token halves, d/16 mma each)
+//   O[16 rows x d]         += P[16 x 16 tokens] . V[16 x d]  (d/8 mma, twice: P's 2-byte head and residual)
+// P's accumulator layout is the A operand's, so it feeds the second product without a transpose.  Each thread
+// holds rows gid and gid + 8 and keeps their online softmax state.
+template <class E, int D>
+struct RowTile {
+  static constexpr int KSTEPS = D / 16, NT = D / 8;
+  uint32_t qa[KSTEPS][4];
+  float o[NT][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows gid, gid + 8
+  int gid, tig, kb_tok, kb_c, vb_tok, vb_c;
+
+  __device__ __forceinline__ void init(const CascadeArgs &a, int lane, int seq_lo, int head_lo, int seq_hi,
+                                       int head_hi) {
+    gid = lane >> 2;
+    tig = lane & 3;
+    const int mi = lane >> 3, mr = lane & 7;
+    kb_tok = 8 * (mi >> 1) + mr, kb_c = mi & 1;  // K rows as the B operand: [tokens 0-7 | 8-15] x [dims lo | hi]
+    vb_tok = 8 * (mi & 1) + mr, vb_c = mi >> 1;  // V rows as the B operand, transposed: two 8-dim column tiles
+    const uint32_t *qlo = reinterpret_cast<const uint32_t *>(a.q + (long long)max(seq_lo, 0) * a.q_seq_stride +
+                                                             (long long)head_lo * D);
+    const uint32_t *qhi = reinterpret_cast<const uint32_t *>(a.q + (long long)max(seq_hi, 0) * a.q_seq_stride +
+                                                             (long long)head_hi * D);
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+      qa[ks][0] = seq_lo >= 0 ? __ldg(qlo + 8 * ks + tig) : 0u;
+      qa[ks][1] = seq_hi >= 0 ? __ldg(qhi + 8 * ks + tig) : 0u;
+      qa[ks][2] = seq_lo >= 0 ? __ldg(qlo + 8 * ks + 4 + tig) : 0u;
+      qa[ks][3] = seq_hi >= 0 ? __ldg(qhi + 8 * ks + 4 + tig) : 0u;
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+  }
+
+  // S = Q K^T from the slot at shared address kt, and the V fragments; the slot may be reused after this
+  __device__ __forceinline__ void scores(uint32_t kt, float (&s)[2][4], uint32_t (&vf)[NT / 2][4]) const {
+    constexpr uint32_t TILE_BYTES = TILE * D * 2;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) s[h2][0] = s[h2][1] = s[h2][2] = s[h2][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+      uint32_t kf[4];
+      ldsm_x4(kf, kt + swizzled(kb_tok, 2 * ks + kb_c));
+      MmaOps<E>::mma(s[0], qa[ks], kf[0], kf[1]);
+      MmaOps<E>::mma(s[1], qa[ks], kf[2], kf[3]);
+    }
+#pragma unroll
+    for (int c2 = 0; c2 < NT / 2; ++c2) ldsm_x4_trans(vf[c2], kt + TILE_BYTES + swizzled(vb_tok, 2 * c2 + vb_c));
+  }
+
+  __device__ __forceinline__ void accumulate(const CascadeArgs &a, const float (&s)[2][4], uint32_t (&vf)[NT / 2][4],
+                                             int nvalid) {
+    // z[h2][0..1]: row gid, tokens 8*h2 + 2tig, +1; z[h2][2..3]: row gid + 8
+    float z[2][4];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) z[h2][k] = 8 * h2 + 2 * tig + (k & 1) < nvalid ? s[h2][k] * a.scale_log2 : -INFINITY;
+    const float c0 = fmaxf(fmaxf(z[0][0], z[0][1]), fmaxf(z[1][0], z[1][1]));
+    const float c1 = fmaxf(fmaxf(z[0][2], z[0][3]), fmaxf(z[1][2], z[1][3]));
+    if (__any_sync(FULL, c0 > m0 + RESCALE_SLACK || c1 > m1 + RESCALE_SLACK)) {
+      float r0 = fmaxf(c0, __shfl_xor_sync(FULL, c0, 1)), r1 = fmaxf(c1, __shfl_xor_sync(FULL, c1, 1));
+      r0 = fmaxf(r0, __shfl_xor_sync(FULL, r0, 2));
+      r1 = fmaxf(r1, __shfl_xor_sync(FULL, r1, 2));
+      const float n0 = fmaxf(m0, r0), n1 = fmaxf(m1, r1);
+      const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);  // 0 on the first tile
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        o[nt][0] *= al0;
+        o[nt][1] *= al0;
+        o[nt][2] *= al1;
+        o[nt][3] *= al1;
+      }
+      l0 *= al0;
+      l1 *= al1;
+      m0 = n0;
+      m1 = n1;
+    }
+    float p[2][4];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      p[h2][0] = exp2f(z[h2][0] - m0);
+      p[h2][1] = exp2f(z[h2][1] - m0);
+      p[h2][2] = exp2f(z[h2][2] - m1);
+      p[h2][3] = exp2f(z[h2][3] - m1);
+    }
+    l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+    l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+    // A operand of P . V: a0 row gid tokens 2tig..; a1 row gid + 8; a2, a3 the same rows, tokens 8 + 2tig..
+    uint32_t ah[4], al[4];
+    MmaOps<E>::split(p[0][0], p[0][1], ah[0], al[0]);
+    MmaOps<E>::split(p[0][2], p[0][3], ah[1], al[1]);
+    MmaOps<E>::split(p[1][0], p[1][1], ah[2], al[2]);
+    MmaOps<E>::split(p[1][2], p[1][3], ah[3], al[3]);
+    if (nvalid < TILE) {  // V rows past the context may hold NaN: zero them (0 * NaN would leak in)
+      const uint32_t m_lo = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
+      const uint32_t m_hi = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
+#pragma unroll
+      for (int c2 = 0; c2 < NT / 2; ++c2) {
+        vf[c2][0] &= m_lo;
+        vf[c2][1] &= m_hi;
+        vf[c2][2] &= m_lo;
+        vf[c2][3] &= m_hi;
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t b0 = vf[nt >> 1][(nt & 1) * 2], b1 = vf[nt >> 1][(nt & 1) * 2 + 1];
+      MmaOps<E>::mma(o[nt], ah, b0, b1);
+      MmaOps<E>::mma(o[nt], al, b0, b1);
+    }
+  }
+
+  // Writes rows gid and gid + 8 (if live) to partial rows row_lo / row_hi (per kv head), as ColumnTile::store.
+  __device__ __forceinline__ void store(const CascadeArgs &a, long long row_lo, long long row_hi, bool live_lo,
+                                        bool live_hi, bool bad_lo, bool bad_hi, bool any_tiles) {
+    float t0 = l0 + __shfl_xor_sync(FULL, l0, 1), t1 = l1 + __shfl_xor_sync(FULL, l1, 1);
+    t0 += __shfl_xor_sync(FULL, t0, 2);
+    t1 += __shfl_xor_sync(FULL, t1, 2);
+    if (tig == 0) {
+      if (live_lo) a.ws_ml[row_lo] = bad_lo ? make_float2(-INFINITY, -1.f) : make_float2(m0, t0);
+      if (live_hi) a.ws_ml[row_hi] = bad_hi ? make_float2(-INFINITY, -1.f) : make_float2(m1, t1);
+    }
+    if (!any_tiles) return;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (live_lo && !bad_lo)
+        *reinterpret_cast<float2 *>(a.ws_acc + row_lo * D + 8 * nt + 2 * tig) = make_float2(o[nt][0], o[nt][1]);
+      if (live_hi && !bad_hi)
+        *reinterpret_cast<float2 *>(a.ws_acc + row_hi * D + 8 * nt + 2 * tig) = make_float2(o[nt][2], o[nt][3]);
+    }
+  }
+};
+
+// One job of the plan, read and checked (the plan lives in the caller's memory).  `per` is the members one
+// warp holds: 8 / G columns for a suffix job's warp, 16 / G rows for a prefix job's row tile.
 struct CascadeJob {
-  int ts, t0, t1, mbase, nm, row0, kind;
-  __device__ __forceinline__ bool load(const CascadeArgs &a, int j, int mpo) {
+  int ts, t0, t1, mbase, nm, row0, kind, split;
+  __device__ __forceinline__ bool load(const CascadeArgs &a, int j, int per) {
     const int *job = a.jobs + (long long)j * CJ_INTS;
     ts = __ldg(job + CJ_SEQ), t0 = __ldg(job + CJ_T0), t1 = __ldg(job + CJ_T1);
     mbase = __ldg(job + CJ_MEMBERS), nm = __ldg(job + CJ_NM), row0 = __ldg(job + CJ_ROW), kind = __ldg(job + CJ_KIND);
+    split = __ldg(job + CJ_SPLIT);
     const bool prefix = j < a.num_prefix_jobs;
-    return ts >= 0 && ts < a.num_seqs && t0 >= 0 && t1 >= t0 && nm >= 1 && mbase >= 0 &&
-           mbase <= a.num_members - nm && row0 >= 0 && row0 <= a.rows_per_head - nm * a.group &&
-           (prefix ? (kind == CJ_PREFIX && nm <= CASCADE_CONSUMERS * mpo)
-                   : (kind == CJ_SUFFIX && nm == 1 && __ldg(a.members + mbase) == ts));
+    const int n_rt = (nm + per - 1) / per;
+    const bool shape_ok = prefix ? (kind == CJ_PREFIX && (split == 1 || split == 2 || split == 4) &&
+                                    nm <= CASCADE_CONSUMERS * per && n_rt * split <= CASCADE_CONSUMERS)
+                                 : (kind == CJ_SUFFIX && split == 1 && nm == 1);
+    return shape_ok && ts >= 0 && ts < a.num_seqs && t0 >= 0 && t1 >= t0 && nm >= 1 && mbase >= 0 &&
+           mbase <= a.num_members - nm && row0 >= 0 && (long long)row0 + (long long)nm * a.group * split <= a.rows_per_head &&
+           (prefix || __ldg(a.members + mbase) == ts);
   }
 };
 
@@ -240,7 +385,7 @@ struct CascadeJob {
 // free.  Blocks after them: CASCADE_CONSUMERS suffix jobs each, one per warp, every warp streaming its own
 // tiles through its own CASCADE_WARP_SLOTS slots and issuing them itself.
 template <class E, int D>
-__global__ void __launch_bounds__(CASCADE_CONSUMERS * 32)
+__global__ void __launch_bounds__(CASCADE_CONSUMERS * 32, CASCADE_MIN_BLOCKS)
     cascade_partial_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                            const CascadeArgs a) {
   constexpr int KSTEPS = D / 16;
@@ -289,7 +434,10 @@ __global__ void __launch_bounds__(CASCADE_CONSUMERS * 32)
       const int t = jb.t0 + i;
       const int phys = win.lookup(row, t * TILE / a.block_size, nblk, lane);
       const int st = i % CASCADE_WARP_SLOTS;
-      if (lane == 0) cascade_issue<D>(a, &tmap_k, &tmap_v, phys, t, h, wring + st * STAGE_BYTES, &wfull[st], &wbad[st]);
+      if (lane == 0) {
+        fence_proxy_async_smem();  // the slot's previous tile was read through the generic proxy
+        cascade_issue<D>(a, &tmap_k, &tmap_v, phys, t, h, wring + st * STAGE_BYTES, &wfull[st], &wbad[st]);
+      }
     };
     for (int i = 0; i < CASCADE_WARP_SLOTS && i < nt; ++i) issue(i);
     ColumnTile<E, D> ct;
@@ -322,22 +470,25 @@ __global__ void __launch_bounds__(CASCADE_CONSUMERS * 32)
     return;
   }
 
-  // ---------------- a prefix job: the block's warps share the ring
+  // ---------------- a prefix job: the block's warps share the ring.  Warp w takes row tile w % n_rt (16 of the
+  // job's member x head rows) and tiles i = w / n_rt (mod split) of the job.
   CascadeJob jb;
-  if (!jb.load(a, (int)blockIdx.x, mpo)) {
+  const int mpr = 16 / G;  // members per row tile
+  if (!jb.load(a, (int)blockIdx.x, mpr)) {
     if (threadIdx.x == 0) atomicOr(&g_status, PA_DEV_ERR_PLAN);
     return;
   }
+  const int n_rt = (jb.nm + mpr - 1) / mpr;
+  const int split = jb.split;
   const int L_lead = __ldg(a.context_lens + jb.ts);
   const bool lead_ok = cascade_context_ok(a, L_lead);
   const bool prefix_short = lead_ok && (long long)jb.t1 * TILE > L_lead;  // the leader does not hold the range
   const int nt = (lead_ok && !prefix_short) ? jb.t1 - jb.t0 : 0;
-  const int n_oct = (jb.nm + mpo - 1) / mpo;  // warps with columns
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int st = 0; st < CASCADE_SLOTS; ++st) {
       mbar_init(&full[st], 1);
-      mbar_init(&empty[st], n_oct);
+      mbar_init(&empty[st], n_rt);  // tile i is read by the n_rt warps of split i % split
       tile_bad[st] = 0;
     }
     // a leader that fails, or does not hold the range, fails the job for every member
@@ -346,56 +497,68 @@ __global__ void __launch_bounds__(CASCADE_CONSUMERS * 32)
     fence_mbar_init();
   }
   __syncthreads();
-  if (warp >= n_oct) return;  // no columns for this warp
+  const int n_warps = n_rt * split;
+  if (warp >= n_warps) return;
+  const int rt = warp % n_rt, sp = warp / n_rt;
   const int *lead_row = a.block_tables + (long long)jb.ts * a.table_stride;
   const int nblk = nt > 0 ? (jb.t1 * TILE + a.block_size - 1) / a.block_size : 0;
-  RowWindow win;
   int issued = 0;
   bool issue_failed = false;
-  // warp 0: issue tiles up to `upto` (inclusive) that are not issued yet; tile `need` and those before it are
-  // waited for, later ones only if their slot is already free.  Returns false if a wait ran out.
+  // warp 0: issue tiles up to `upto` (inclusive) that are not issued yet; tiles up to `need` are waited for,
+  // later ones only if their slot is already free.  Lane k takes the k-th next tile, so a run of free slots is
+  // filled by one round of copies.  Returns false if a wait ran out.
   auto refill = [&](int need, int upto) {
     while (issued < nt && issued <= upto) {
-      const int jt = issued, st = jt % CASCADE_SLOTS;
-      if (jt >= CASCADE_SLOTS) {
-        const uint32_t par = (uint32_t)(jt / CASCADE_SLOTS - 1) & 1u;
-        bool free_slot;
-        if (jt <= need) {
-          free_slot = __all_sync(FULL, mbar_wait_bounded(&empty[st], par, a.wait_limit_ns));
-          if (!free_slot) return false;
-        } else {
-          free_slot = __all_sync(FULL, mbar_try_wait(&empty[st], par));
-          if (!free_slot) return true;
-        }
+      const int jt = issued + lane;
+      bool ready = jt < nt && jt <= upto;
+      if (ready && jt >= CASCADE_SLOTS)
+        ready = mbar_try_wait(&empty[jt % CASCADE_SLOTS], (uint32_t)(jt / CASCADE_SLOTS - 1) & 1u);
+      const unsigned run = __ballot_sync(FULL, ready);
+      const int c = run == FULL ? 32 : __ffs(~run) - 1;  // lanes 0 .. c-1 issue
+      if (c == 0) {
+        if (issued > need) return true;
+        const int st = issued % CASCADE_SLOTS;  // a tile that is needed now: wait for its slot
+        if (!__all_sync(FULL, mbar_wait_bounded(&empty[st], (uint32_t)(issued / CASCADE_SLOTS - 1) & 1u, a.wait_limit_ns)))
+          return false;
+        continue;
       }
-      const int t = jb.t0 + jt;
-      const int phys = win.lookup(lead_row, t * TILE / a.block_size, nblk, lane);
-      if (lane == 0) cascade_issue<D>(a, &tmap_k, &tmap_v, phys, t, h, ring + st * STAGE_BYTES, &full[st], &tile_bad[st]);
+      if (lane < c) {
+        const int t = jb.t0 + jt;
+        const int phys = __ldg(lead_row + t * TILE / a.block_size);  // an entry below nblk
+        fence_proxy_async_smem();  // the freed slot was read through the generic proxy
+        cascade_issue<D>(a, &tmap_k, &tmap_v, phys, t, h, ring + (jt % CASCADE_SLOTS) * STAGE_BYTES,
+                         &full[jt % CASCADE_SLOTS], &tile_bad[jt % CASCADE_SLOTS]);
+      }
       __syncwarp();
-      ++issued;
+      issued += c;
     }
     return true;
   };
-  if (warp == 0) {
+  // this lane's rows gid and gid + 8 of the row tile: member rt * mpr + r / G, head r % G
+  const int gid = lane >> 2;
+  const int r_lo = gid, r_hi = gid + 8;
+  const int ml_lo = rt * mpr + r_lo / G, ml_hi = rt * mpr + r_hi / G;
+  const bool live_lo = r_lo < mpr * G && ml_lo < jb.nm, live_hi = r_hi < mpr * G && ml_hi < jb.nm;
+  RowTile<E, D> rtile;
+  {
+    int m_lo = live_lo ? __ldg(a.members + jb.mbase + ml_lo) : -1;
+    int m_hi = live_hi ? __ldg(a.members + jb.mbase + ml_hi) : -1;
+    if (m_lo >= a.num_seqs) m_lo = -1;  // flagged by the member checks below
+    if (m_hi >= a.num_seqs) m_hi = -1;
+    rtile.init(a, lane, m_lo, h * G + r_lo % G, m_hi, h * G + r_hi % G);
+  }
+  if (warp == 0) {  // the first tiles, while the Q loads above are in flight
     if (lane == 0) {
       prefetch_tensor_map(&tmap_k);
       prefetch_tensor_map(&tmap_v);
     }
     refill(-1, CASCADE_SLOTS - 1);
   }
-  const int mo = warp * mpo;  // the warp's first member
-  ColumnTile<E, D> ct;
-  {
-    const int gid = lane >> 2;
-    const bool live = gid < mpo * G && mo + gid / G < jb.nm;
-    int m = live ? __ldg(a.members + jb.mbase + mo + gid / G) : -1;
-    if (m >= a.num_seqs) m = -1;  // flagged by the member checks below
-    ct.init(a, lane, m, h * G + (live ? gid % G : 0));
-  }
   bool bad = false;
-  for (int i = 0; i < nt; ++i) {
+  int done = 0;  // tiles this warp consumed
+  for (int i = sp; i < nt; i += split) {
     const int st = i % CASCADE_SLOTS;
-    if (warp == 0 && !issue_failed && !refill(i, i + CASCADE_SLOTS - 1)) {
+    if (warp == 0 && !issue_failed && !refill(i + split - 1, i + CASCADE_SLOTS - 1)) {
       if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_TIMEOUT);
       issue_failed = true;
     }
@@ -410,12 +573,13 @@ __global__ void __launch_bounds__(CASCADE_CONSUMERS * 32)
       if (lane == 0) atomicOr(&g_status, PA_DEV_ERR_BLOCK_ID);
       bad = true;
     }
-    float sc[4];
-    uint32_t vf[KSTEPS][4];
-    if (!bad) ct.scores(smem_addr(ring + st * STAGE_BYTES), sc, vf);
+    float sc[2][4];
+    uint32_t vf[RowTile<E, D>::NT / 2][4];
+    if (!bad) rtile.scores(smem_addr(ring + st * STAGE_BYTES), sc, vf);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the slot
-    if (!bad) ct.accumulate(a, sc, vf, TILE);
+    if (!bad) rtile.accumulate(a, sc, vf, TILE);
+    ++done;
   }
   if (warp == 0) {
     // every member's table must name the leader's blocks over the job's range, and its context must hold it
@@ -439,13 +603,12 @@ __global__ void __launch_bounds__(CASCADE_CONSUMERS * 32)
       mbar_wait_bounded(&full[i % CASCADE_SLOTS], (uint32_t)(i / CASCADE_SLOTS) & 1u, a.wait_limit_ns);
     }
   }
-  asm volatile("bar.sync 1, %0;" ::"r"((uint32_t)n_oct * 32u) : "memory");  // member_bad is final
+  asm volatile("bar.sync 1, %0;" ::"r"((uint32_t)n_warps * 32u) : "memory");  // member_bad is final
   const uint32_t mbad = (uint32_t)*member_bad;
-  uint32_t bad_cols = bad ? 0xffu : 0u;
-  for (int c = 0; c < 8; ++c)
-    if ((mbad >> min(31, mo + c / G)) & 1u) bad_cols |= 1u << c;
-  const int ncols = min(mpo, jb.nm - mo) * G;
-  ct.store(a, (long long)h * a.rows_per_head + jb.row0 + (long long)mo * G, ncols, bad_cols, nt > 0);
+  // rows of split sp: row0 + sp * nm * G + member * G + head
+  const long long base = (long long)h * a.rows_per_head + jb.row0 + (long long)sp * jb.nm * G + (long long)rt * mpr * G;
+  rtile.store(a, base + r_lo, base + r_hi, live_lo, live_hi, bad || ((mbad >> min(31, ml_lo)) & 1u),
+              bad || ((mbad >> min(31, ml_hi)) & 1u), done > 0);
 }
 
 // One warp per (sequence, query head).  Pieces with l = 0 (no tiles) take no part; a piece with l < 0 (a

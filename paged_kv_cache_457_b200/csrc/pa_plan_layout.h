@@ -11,12 +11,15 @@ constexpr int CJ_T0 = 1;       // first 16-token tile
 constexpr int CJ_T1 = 2;       // tile bound (exclusive); a suffix job also stops at its sequence's length
 constexpr int CJ_MEMBERS = 3;  // first entry of the job's members in the member list
 constexpr int CJ_NM = 4;       // members: sequences whose query heads are the job's columns
-constexpr int CJ_ROW = 5;      // first partial row of the job (per kv head); member i, head j -> row + i*G + j
+constexpr int CJ_ROW = 5;      // first partial row of the job (per kv head); split s, member i, head j ->
+                               // row + (s * members + i) * G + j
 constexpr int CJ_KIND = 6;     // CJ_PREFIX or CJ_SUFFIX
+constexpr int CJ_SPLIT = 7;    // prefix job: its tiles are dealt round-robin to `split` warp sets (1, 2 or 4), each
+                               // leaving its own partial rows; suffix job: 1
 constexpr int CJ_PREFIX = 0, CJ_SUFFIX = 1;
-constexpr int CASCADE_CONSUMERS = 4;  // warps per block of the partial kernel: a prefix job's column sets, or
-                                      // one suffix job each
+constexpr int CASCADE_CONSUMERS = 4;  // warps per block of the partial kernel: a prefix job's row tiles (16
+                                      // member x head rows each) times its split, or one suffix job each
 constexpr int CASCADE_TILE = 16;      // tokens per tile
-constexpr int CASCADE_DEFAULT_CHUNK_TOKENS = 256;
+constexpr int CASCADE_DEFAULT_CHUNK_TOKENS = 128;
 
 }  // namespace pa

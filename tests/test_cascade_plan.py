@@ -8,7 +8,7 @@ import pytest
 
 import paged_kv_cache_457_b200 as pa
 
-CJ = 8  # ints per job: seq, t0, t1, member offset, members, row, kind, 0
+CJ = 8  # ints per job: seq, t0, t1, member offset, members, row, kind, split
 PREFIX, SUFFIX = 0, 1
 
 
@@ -94,27 +94,34 @@ def check_plan(plan, S, G, bs, mcl, prefix_of, lead_of, chunk):
     kinds = list(jobs[:, 6])
     assert kinds == sorted(kinds) and kinds.count(PREFIX) == info.num_prefix_jobs, "prefix jobs come first"
     row_owner = {}
-    for j, (seq, t0, t1, mfirst, nm, row, kind, zero) in enumerate(jobs):
-        assert zero == 0 and kind in (PREFIX, SUFFIX) and 0 <= t0 < t1 and t1 - t0 <= chunk // 16
-        assert 1 <= nm <= 4 * (8 // G) and 0 <= mfirst and mfirst + nm <= info.num_members
-        assert 0 <= row and row + nm * G <= info.rows_per_head
-        for i in range(nm):
-            m = int(members[mfirst + i])
-            for h in range(G):
-                assert (row + i * G + h) not in row_owner, "partial rows overlap"
-                row_owner[row + i * G + h] = (j, m)
-            if kind == SUFFIX:
-                assert nm == 1 and m == seq
-            else:
-                assert lead_of[m] == seq and t1 <= prefix_of[m]
+    for j, (seq, t0, t1, mfirst, nm, row, kind, split) in enumerate(jobs):
+        assert kind in (PREFIX, SUFFIX) and 0 <= t0 < t1 and t1 - t0 <= chunk // 16
+        if kind == SUFFIX:
+            assert nm == 1 and split == 1
+        else:
+            n_rt = -(-nm // (16 // G))  # row tiles of 16 (member, head) rows
+            assert 1 <= nm <= 4 * (16 // G) and split == {1: 4, 2: 2}.get(n_rt, 1) and n_rt * split <= 4
+        assert 0 <= mfirst and mfirst + nm <= info.num_members
+        assert 0 <= row and row + nm * G * split <= info.rows_per_head
+        for sp in range(split):
+            for i in range(nm):
+                m = int(members[mfirst + i])
+                for h in range(G):
+                    r = row + (sp * nm + i) * G + h
+                    assert r not in row_owner, "partial rows overlap"
+                    row_owner[r] = (j, m, sp)
+                if kind == SUFFIX:
+                    assert m == seq
+                else:
+                    assert lead_of[m] == seq and t1 <= prefix_of[m]
     assert len(row_owner) == info.rows_per_head
     for s in range(S):
         covered = []
         for r in rows[offs[s]:offs[s + 1]]:
-            j, m = row_owner[int(r)]
+            j, m, sp = row_owner[int(r)]
             assert m == s, "a piece row of another sequence"
-            covered += list(range(jobs[j][1], jobs[j][2]))
-        assert covered == list(range(max(max_tiles, prefix_of[s]))), f"sequence {s}: tiles {covered}"
+            covered += list(range(jobs[j][1] + sp, jobs[j][2], jobs[j][7]))
+        assert sorted(covered) == list(range(max(max_tiles, prefix_of[s]))), f"sequence {s}: tiles {covered}"
 
 
 @pytest.mark.parametrize("hq,hkv", [(32, 8), (8, 8), (16, 8), (24, 8), (8, 1), (6, 2)])
@@ -134,19 +141,21 @@ def test_cascade_plan_covers_every_tile_once(hq, hkv, chunk, seed):
         for m in mem:
             prefix_of[m] = int(g.prefix_blocks[i]) * bs // 16
             lead_of[m] = int(mem[0])
-    check_plan(plan, S, hq // hkv, bs, mcl, prefix_of, lead_of, chunk or 256)
+    check_plan(plan, S, hq // hkv, bs, mcl, prefix_of, lead_of, chunk or 128)
     assert plan.info.num_seqs == S and plan.info.max_context_len == mcl
 
 
 def test_cascade_plan_large_group_splits_columns():
-    """A group of 70 members with 4 heads per kv head: column sets of 8 members (4 warps x 2)."""
+    """A group of 70 members with 4 heads per kv head: jobs of 16 members (4 row tiles of 4 members x 4 heads,
+    no split) and one of 6 (2 row tiles, its tiles dealt to 2 warp sets)."""
     S, bs = 70, 16
     g = pa.PrefixGroups(np.array([0, S], np.int32), np.arange(S, dtype=np.int32), np.array([40], np.int32))
     plan = pa.cascade_plan(S, 32, 8, bs, 700, g, chunk_tokens=256)
     jobs, *_ = pieces_of(plan, S)
     pre = jobs[jobs[:, 6] == PREFIX]
-    assert sorted(set(pre[:, 4].tolist())) == [6, 8]  # 8 full column sets and one of 6
-    assert pre.shape[0] == 9 * 3  # 40 blocks = 40 tiles: chunks of 16, 16, 8
+    assert sorted(set(pre[:, 4].tolist())) == [6, 16]
+    assert sorted(set(zip(pre[:, 4].tolist(), pre[:, 7].tolist()))) == [(6, 2), (16, 1)]
+    assert pre.shape[0] == 5 * 3  # 40 blocks = 40 tiles: chunks of 16, 16, 8
     check_plan(plan, S, 4, bs, 700, [40] * S, [0] * S, 256)
 
 
