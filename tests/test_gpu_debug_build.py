@@ -21,6 +21,8 @@ CASES = [
     "tests/test_gpu_parity.py::test_many_short_sequences",
     "tests/test_gpu_parity.py::test_shared_prefix_tables",
     "tests/test_gpu_parity.py::test_shared_prefix_bad_block_zeroes_only_its_sequence",
+    "tests/test_gpu_cascade.py::test_cascade_planted_groups",
+    "tests/test_gpu_cascade.py::test_cascade_device_checks",
     "tests/test_gpu_errors.py",
     "tests/test_gpu_properties.py",
     "tests/test_gpu_launch_config.py",
