@@ -98,13 +98,16 @@ def step_bytes(wl, st):
     return kv, kv + qo + 4 * nblk + 4 * st.num_seqs
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, path: str | None = None):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary, or (None, reason)
-    when the kernel sources changed since the capture or the workload was not captured."""
+    when the kernel sources changed since the capture or the workload was not captured.  ``path``
+    selects a record of another decode path (``"cascade"``), kept under that key with its own sources."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
             rec = json.load(f)
+        if path is not None:
+            rec = rec[path]
         h = hashlib.sha256()
         for rel in rec["kernel_sources"]:
             with open(os.path.join(ROOT, rel), "rb") as f:
@@ -992,8 +995,7 @@ def main():
         value_distinct = job_rate_gbs(uniq_kv, world, args.steps, elapsed_ms)
         peak, peak_kind = measured_peak()
         achieved = alg_unique / (dec_ms / 1e3) / 1e9
-        traffic, traffic_note = recorded_traffic(wl.name) if not use_cascade else (
-            None, "no ncu capture of the cascade kernels")
+        traffic, traffic_note = recorded_traffic(wl.name, "cascade" if use_cascade else None)
         shared = uniq_kv != kv_b
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -1007,7 +1009,11 @@ def main():
             "config": {"workload": wl.name, "description": wl.description, "num_seqs": st.num_seqs,
                        "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                        "block_size": wl.block_size, "max_context_len": mcl,
-                       "split": f"chunks of {part} tokens" if part else "balanced (one chunk of tiles per warp)",
+                       "split": (f"cascade plan: {plan.info.num_prefix_jobs} prefix jobs (a group's shared tiles), "
+                                 f"{plan.info.num_jobs - plan.info.num_prefix_jobs} suffix jobs, "
+                                 f"{plan.info.num_pieces} partial states to combine") if use_cascade else
+                                (f"chunks of {part} tokens" if part else
+                                 "balanced tile stream cut into chunks, one queue of chunks shared by the warps"),
                        "kv_bytes_per_step": kv_b, "distinct_kv_bytes_per_step": uniq_kv,
                        "parallelism": f"dp{world} (independent batches per GPU)",
                        "timing": ("per-step CUDA events, L2 flushed before each step" if flush else
