@@ -122,6 +122,13 @@ def recorded_traffic(workload: str, path: str | None = None):
         return None, f"no traffic record ({type(e).__name__})"
 
 
+def cascade_wanted(mode: str, num_groups: int, partition_tokens: int) -> bool:
+    """Whether the decode step runs through pa_decode_cascade: always with ``on``; with ``auto`` when the
+    host found prefix groups in the step's tables and no fixed partition was asked for (a partition
+    length is a parameter of pa_decode's split, which the cascade plan does not take)."""
+    return mode == "on" or (mode == "auto" and num_groups > 0 and partition_tokens == 0)
+
+
 def max_over_ranks(values, device=None):
     """Elementwise maximum of per-rank timings (ms) over all ranks; identity on one rank."""
     import torch
@@ -751,7 +758,7 @@ def main():
     # Shared leading blocks: the host finds the groups from the step's tables (as a scheduler would) and the
     # cascade path reads each group's shared tiles once.
     groups = pa.find_prefix_groups(st.block_tables, st.context_lens, wl.block_size)
-    use_cascade = args.cascade == "on" or (args.cascade == "auto" and groups.num_groups > 0 and part == 0)
+    use_cascade = cascade_wanted(args.cascade, groups.num_groups, part)
     if use_cascade:
         plan = pa.cascade_plan(st.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.block_size, mcl, groups)
         plan_dev = plan.to(device)

@@ -119,3 +119,47 @@ def test_shared_prefix_distinct_bytes_below_logical():
     kv, _ = bench.step_bytes(wl, st)
     uniq = W.unique_kv_bytes(st, wl.num_kv_heads, wl.head_dim, wl.block_size)
     assert uniq < kv / 3  # 8 tables name each prefix block
+
+
+def test_cascade_traffic_record_has_its_own_sources(tmp_path, monkeypatch):
+    import hashlib
+    fake = tmp_path / "profiles"
+    fake.mkdir()
+    (tmp_path / "a.cuh").write_text("split kernel")
+    (tmp_path / "c.cuh").write_text("cascade kernel v1")
+    rec = {"kernel_sources": ["a.cuh"], "kernel_sources_sha256": hashlib.sha256(b"split kernel").hexdigest(),
+           "workloads": {"w": {"kernel": "split", "dram_bytes_per_launch": 10, "how": "t"}},
+           "cascade": {"kernel_sources": ["c.cuh"],
+                       "kernel_sources_sha256": hashlib.sha256(b"cascade kernel v1").hexdigest(),
+                       "workloads": {"w": {"kernel": "partial", "dram_bytes_per_launch": 20, "how": "t"}}}}
+    (fake / "decode_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("w")[0] == 10
+    assert bench.recorded_traffic("w", "cascade")[0] == 20
+    (tmp_path / "c.cuh").write_text("cascade kernel v2")  # only the cascade record goes stale
+    assert bench.recorded_traffic("w", "cascade") == (None, "kernel changed since the ncu capture")
+    assert bench.recorded_traffic("w")[0] == 10
+    assert bench.recorded_traffic("w", "missing")[0] is None
+
+
+def test_committed_cascade_traffic_record_matches_the_sources():
+    val, note = bench.recorded_traffic("shared_prefix_step", "cascade")
+    assert val is not None, note
+    wl = W.shared_prefix()
+    uniq = W.unique_kv_bytes(wl.steps[0], wl.num_kv_heads, wl.head_dim, wl.block_size)
+    assert uniq < val < 1.1 * uniq  # the shared tiles cross HBM once per group
+
+
+def test_bench_decodes_through_the_cascade_only_when_groups_are_found():
+    import paged_kv_cache_457_b200 as pa
+    wl = W.shared_prefix()
+    st = wl.steps[0]
+    g = pa.find_prefix_groups(st.block_tables, st.context_lens, wl.block_size)
+    assert g.num_groups == 8 and set(np.diff(g.offsets).tolist()) == {8} and set(g.prefix_blocks.tolist()) == {64}
+    assert bench.cascade_wanted("auto", g.num_groups, 0)
+    assert not bench.cascade_wanted("auto", g.num_groups, 256)  # a fixed partition is pa_decode's parameter
+    assert not bench.cascade_wanted("off", g.num_groups, 0)
+    tiny = W.tiny()
+    g0 = pa.find_prefix_groups(tiny.steps[0].block_tables, tiny.steps[0].context_lens, tiny.block_size)
+    assert g0.num_groups == 0 and not bench.cascade_wanted("auto", 0, 0)
+    assert bench.cascade_wanted("on", 0, 0)
