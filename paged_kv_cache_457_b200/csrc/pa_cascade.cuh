@@ -611,15 +611,48 @@ __global__ void __launch_bounds__(CASCADE_CONSUMERS * 32, CASCADE_MIN_BLOCKS)
               bad || ((mbad >> min(31, ml_hi)) & 1u), done > 0);
 }
 
+// Partial rows [i0, i0 + MB) of a 32-piece window whose lane p holds piece p's row r and range flag bad, for
+// query head hh of the kv head whose rows start at head_rows: lane l takes dims [l * DPL, (l + 1) * DPL).  Rows
+// at or past nw, or out of range, are not read (zeros).
+template <int D, int MB>
+__device__ __forceinline__ void cascade_load_rows(const CascadeArgs &a, float (&t)[MB][D / 32], long long head_rows,
+                                                  int hh, int r, bool bad, int i0, int nw, int lane) {
+  constexpr int DPL = D / 32;
+#pragma unroll
+  for (int i = 0; i < MB; ++i) {
+    const int ri = __shfl_sync(FULL, r, (i0 + i) & 31);
+    const bool bi = __shfl_sync(FULL, bad ? 1 : 0, (i0 + i) & 31) != 0;
+    const bool use = i0 + i < nw && !bi;  // warp-uniform
+    const float *src = a.ws_acc + (head_rows + ri + hh) * D + lane * DPL;
+    if constexpr (DPL == 4) {
+      const float4 v = use ? __ldg(reinterpret_cast<const float4 *>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      t[i][0] = v.x;
+      t[i][1] = v.y;
+      t[i][2] = v.z;
+      t[i][3] = v.w;
+    } else {
+      const float2 v = use ? __ldg(reinterpret_cast<const float2 *>(src)) : make_float2(0.f, 0.f);
+      t[i][0] = v.x;
+      t[i][1] = v.y;
+    }
+  }
+}
+
 // One warp per (sequence, query head).  Pieces with l = 0 (no tiles) take no part; a piece with l < 0 (a
 // job that failed and set its own status bit) zeroes the row.  A context outside [0, min(table capacity, max_context_len)] gives a zero row
 // and its status bit, as in pa_decode.
+//
+// Memory trips.  Behind the partial kernel (num_jobs > 0) the length, the piece offsets and the first 32 piece
+// rows are read before the grid-dependency wait: they are inputs of the call, which the partial kernel does not
+// write, and that kernel triggers this launch only after its own wait, so every earlier write in the stream is
+// complete by then.  After the wait, the pieces' (m, l) and the partial rows of the first MB pieces are requested
+// in one trip.  Without a partial kernel the wait comes first, as the inputs may come from the previous kernel.
 template <class E, int D>
 __global__ void __launch_bounds__(256) cascade_combine_kernel(const CascadeArgs a) {
   constexpr int DPL = D / 32;  // dims per lane
   constexpr int MB = 8;        // partial rows requested together
-  grid_dependency_wait();      // the partial kernel's rows
-  grid_launch_dependents();
+  const bool after_partial = a.num_jobs > 0;
+  if (!after_partial) grid_dependency_wait();  // the inputs may come from the previous kernel in the stream
   const int lane = threadIdx.x & 31;
   const long long w = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (w >= (long long)a.num_seqs * a.num_q_heads) return;
@@ -627,22 +660,40 @@ __global__ void __launch_bounds__(256) cascade_combine_kernel(const CascadeArgs 
   const int hq = (int)(w - (long long)s * a.num_q_heads);
   const int h = hq / a.group, hh = hq - h * a.group;
   const long long head_rows = (long long)h * a.rows_per_head;
+  const int L = __ldg(a.context_lens + s);
+  const int p0 = __ldg(a.piece_offsets + s), p1 = __ldg(a.piece_offsets + s + 1);
+  const bool ctx_ok = cascade_context_ok(a, L);
+  bool err = ctx_ok && L > 0 && !(p0 >= 0 && p0 <= p1 && p1 <= a.num_pieces);  // plan indices out of range
+  const int n = ctx_ok && L > 0 && !err ? p1 - p0 : 0;
+  // the first window's pieces: lane p holds piece p's row and whether it lies inside the workspace
+  int r0 = 0;
+  bool bad0 = false;
+  if (lane < n) {
+    r0 = __ldg(a.piece_rows + p0 + lane);
+    bad0 = r0 < 0 || r0 > a.rows_per_head - a.group;
+  }
+  if (after_partial) grid_dependency_wait();  // the partial kernel's rows
+  grid_launch_dependents();
+
   float o[DPL];
 #pragma unroll
   for (int k = 0; k < DPL; ++k) o[k] = 0.f;
-  const int L = __ldg(a.context_lens + s);
-  if (!cascade_context_ok(a, L)) {
+  if (!ctx_ok) {
     if (lane == 0 && hq == 0)
       atomicOr(&g_status, (L < 0 || (long long)L > (long long)a.table_stride * a.block_size) ? PA_DEV_ERR_CONTEXT
                                                                                             : PA_DEV_ERR_CONTEXT_HINT);
   } else if (L > 0) {
-    const int p0 = __ldg(a.piece_offsets + s), p1 = __ldg(a.piece_offsets + s + 1);
-    bool err = !(p0 >= 0 && p0 <= p1 && p1 <= a.num_pieces);  // plan indices out of range
-    bool failed = false;                                       // a piece whose job flagged its own error
-    const int n = err ? 0 : p1 - p0;
+    // one trip: the first window's (m, l) and the first MB partial rows
+    float2 ml0 = make_float2(-INFINITY, 0.f);
+    if (lane < n && !bad0) ml0 = __ldg(a.ws_ml + head_rows + r0 + hh);
+    const int nw0 = min(32, n);
+    float t[MB][DPL];
+    cascade_load_rows<D, MB>(a, t, head_rows, hh, r0, bad0, 0, nw0, lane);
     // pass 1: the maximum over the pieces with tokens, and whether any piece failed
-    float M = -INFINITY;
-    for (int p = lane; p < n; p += 32) {
+    bool failed = lane < n && !bad0 && ml0.y < 0.f;  // a piece whose job flagged its own error
+    err = err || (lane < n && bad0);
+    float M = lane < n && !bad0 && ml0.y > 0.f ? ml0.x : -INFINITY;
+    for (int p = 32 + lane; p < n; p += 32) {
       const int r = __ldg(a.piece_rows + p0 + p);
       if (r < 0 || r > a.rows_per_head - a.group) {
         err = true;
@@ -662,37 +713,24 @@ __global__ void __launch_bounds__(256) cascade_combine_kernel(const CascadeArgs 
       float l = 0.f;
       for (int base = 0; base < n; base += 32) {
         const int p = base + lane;
-        int r = 0;
-        float wt = 0.f, lp = 0.f;
-        if (p < n) {
-          r = __ldg(a.piece_rows + p0 + p);
-          const float2 ml = __ldg(a.ws_ml + head_rows + r + hh);
-          if (ml.y > 0.f) {
-            wt = exp2f(ml.x - M);
-            lp = ml.y;
+        int r = r0;
+        float2 ml = ml0;
+        if (base > 0) {
+          r = 0;
+          ml = make_float2(-INFINITY, 0.f);
+          if (p < n) {
+            r = __ldg(a.piece_rows + p0 + p);
+            ml = __ldg(a.ws_ml + head_rows + r + hh);
           }
+        }
+        float wt = 0.f, lp = 0.f;
+        if (p < n && ml.y > 0.f) {
+          wt = exp2f(ml.x - M);
+          lp = ml.y;
         }
         const int nw = min(32, n - base);
         for (int i0 = 0; i0 < nw; i0 += MB) {
-          float t[MB][DPL];
-#pragma unroll
-          for (int i = 0; i < MB; ++i) {
-            const int ri = __shfl_sync(FULL, r, (i0 + i) & 31);
-            const float wi = __shfl_sync(FULL, wt, (i0 + i) & 31);
-            const bool use = i0 + i < nw && wi > 0.f;  // warp-uniform
-            const float *src = a.ws_acc + (head_rows + ri + hh) * D + lane * DPL;
-            if constexpr (DPL == 4) {
-              const float4 v = use ? __ldg(reinterpret_cast<const float4 *>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
-              t[i][0] = v.x;
-              t[i][1] = v.y;
-              t[i][2] = v.z;
-              t[i][3] = v.w;
-            } else {
-              const float2 v = use ? __ldg(reinterpret_cast<const float2 *>(src)) : make_float2(0.f, 0.f);
-              t[i][0] = v.x;
-              t[i][1] = v.y;
-            }
-          }
+          if (base > 0 || i0 > 0) cascade_load_rows<D, MB>(a, t, head_rows, hh, r, false, i0, nw, lane);
 #pragma unroll
           for (int i = 0; i < MB; ++i) {
             const float wi = __shfl_sync(FULL, wt, (i0 + i) & 31);
