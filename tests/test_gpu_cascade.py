@@ -199,3 +199,31 @@ def test_cascade_device_checks():
     lens[19] = st.max_context_len + 1  # a member of group 0 (not its first) above the call's bound
     assert lens[19] <= tables.shape[1] * wl.block_size
     check([19], pa.DEV_ERR_CONTEXT_HINT, tables, lens, mcl=st.max_context_len)
+
+
+def test_cascade_without_jobs_runs_the_combine_alone():
+    """A call bounded at max_context_len 0 has no jobs, so the combine kernel runs alone, right behind the
+    kernel that wrote the lengths (it waits for that kernel before reading them).  Empty contexts give zero
+    rows and no status bit; a context above the bound gives a zero row and PA_DEV_ERR_CONTEXT_HINT."""
+    import paged_kv_cache_457_b200 as pa
+    wl = W.custom(seed=3, num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=64, block_size=16, lens=[5, 1, 9, 3],
+                  dtype="fp16")
+    st = wl.steps[0]
+    dev = DeviceState(wl)
+    plan = pa.cascade_plan(4, 8, 2, 16, 0)
+    assert plan.info.num_jobs == 0
+    q = to_dev(st.q, "fp16")
+    tables = to_dev_index(st.block_tables)
+    plan_dev = plan.to("cuda")
+    lens = torch.full((4,), 7, dtype=torch.int32, device="cuda")
+    out = torch.full_like(q, float("nan"))
+    pa.device_status()
+    lens.zero_()  # the kernel just before the call writes the lengths
+    pa.decode_cascade(q, dev.k_cache, dev.v_cache, tables, lens, wl.scale, plan, plan_dev, out=out)
+    assert pa.device_status() == 0
+    assert not np.any(host_bits(out))
+    lens.copy_(torch.tensor([0, 3, 0, 0], dtype=torch.int32))
+    out.fill_(float("nan"))
+    pa.decode_cascade(q, dev.k_cache, dev.v_cache, tables, lens, wl.scale, plan, plan_dev, out=out)
+    assert pa.device_status() == pa.DEV_ERR_CONTEXT_HINT
+    assert not np.any(host_bits(out))
