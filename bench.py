@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--cascade", default="auto", choices=["auto", "on", "off"],
                     help="decode through pa_decode_cascade (prefix groups found on the host from the step's tables); "
                          "auto: when the batch has groups and no fixed partition is asked for")
+    ap.add_argument("--cascade-chunk", type=int, default=0,
+                    help="tokens per cascade job along the context (0: the library's default, 320)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0,
@@ -760,7 +762,8 @@ def main():
     groups = pa.find_prefix_groups(st.block_tables, st.context_lens, wl.block_size)
     use_cascade = cascade_wanted(args.cascade, groups.num_groups, part)
     if use_cascade:
-        plan = pa.cascade_plan(st.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.block_size, mcl, groups)
+        plan = pa.cascade_plan(st.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.block_size, mcl, groups,
+                               chunk_tokens=args.cascade_chunk)
         plan_dev = plan.to(device)
         cws = torch.empty(max(pa.cascade_workspace_size(plan, wl.head_dim), 16), dtype=torch.uint8, device=device)
 

@@ -374,7 +374,7 @@ int pa_find_prefix_groups(const int32_t *block_tables, const int32_t *context_le
  * must hold at least group_prefix_blocks[g] * block_size tokens, and
  * group_prefix_blocks[g] * block_size <= max_context_len.  num_q_heads /
  * num_kv_heads must be at most 8 (PA_ERR_UNSUPPORTED otherwise).
- * chunk_tokens: tokens per job along the context, 0 = 128, else a positive
+ * chunk_tokens: tokens per job along the context, 0 = 320, else a positive
  * multiple of 16 (PA_ERR_PARTITION).  Fills *info; writes the plan
  * (info->plan_ints int32) to `plan` unless it is NULL (a size query).
  * plan_capacity (entries) smaller than needed -> PA_ERR_WORKSPACE, with

@@ -141,7 +141,7 @@ def test_cascade_plan_covers_every_tile_once(hq, hkv, chunk, seed):
         for m in mem:
             prefix_of[m] = int(g.prefix_blocks[i]) * bs // 16
             lead_of[m] = int(mem[0])
-    check_plan(plan, S, hq // hkv, bs, mcl, prefix_of, lead_of, chunk or 128)
+    check_plan(plan, S, hq // hkv, bs, mcl, prefix_of, lead_of, chunk or 320)
     assert plan.info.num_seqs == S and plan.info.max_context_len == mcl
 
 
