@@ -1023,6 +1023,8 @@ def main():
                                  f"{plan.info.num_jobs - plan.info.num_prefix_jobs} suffix jobs, "
                                  f"{plan.info.num_pieces} partial states to combine") if use_cascade else
                                 (f"chunks of {part} tokens" if part else
+                                 "one block per (sequence, kv head) segment, no workspace (small batch)"
+                                 if ws_bytes == 0 else
                                  "balanced tile stream cut into chunks, one queue of chunks shared by the warps"),
                        "kv_bytes_per_step": kv_b, "distinct_kv_bytes_per_step": uniq_kv,
                        "parallelism": f"dp{world} (independent batches per GPU)",
