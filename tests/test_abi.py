@@ -157,3 +157,52 @@ def test_host_validation_of_block_copies(lib):
 def test_status_strings_cover_new_codes(lib):
     for code in (-10, -11):
         assert lib.pa_status_string(code) != b"unknown status"
+
+
+def _cascade(lib, info_over=None, **over):
+    """pa_decode_cascade on fake aligned pointers with a consistent host-built plan (2 sequences, 4 query /
+    2 kv heads, block 16, max_context_len 40, no groups); `info_over` edits the plan's sizes."""
+    import ctypes
+    from paged_kv_cache_457_b200.cascade import CascadeInfo
+    plan = pa.cascade_plan(2, 4, 2, 16, 40)
+    info = CascadeInfo.from_buffer_copy(plan.info)
+    for k, v in (info_over or {}).items():
+        setattr(info, k, v)
+    args = dict(q=16, k=16, v=16, bt=16, cl=16, scale=0.1, out=16, d=128, nb=10, mb=4, qs=512, os_=512, dtype=1,
+                plan=16, ws=256, wsb=1 << 20, stream=None)
+    args.update(over)
+    return lib.pa_decode_cascade(args["q"], args["k"], args["v"], args["bt"], args["cl"], args["scale"], args["out"],
+                                 args["d"], args["nb"], args["mb"], args["qs"], args["os_"], args["dtype"], args["plan"],
+                                 ctypes.byref(info), args["ws"], args["wsb"], args["stream"])
+
+
+def test_host_validation_of_cascade_decode(lib):
+    # every call below fails validation (or has no sequences) before any CUDA call
+    assert _cascade(lib, d=96) == -5
+    assert _cascade(lib, dtype=3) == -2
+    assert _cascade(lib, info_over={"num_q_heads": 5}) == -6
+    assert _cascade(lib, info_over={"num_q_heads": 18}) == -5  # 9 query heads per kv head
+    assert _cascade(lib, info_over={"block_size": 8}) == -5
+    assert _cascade(lib, info_over={"max_context_len": -1}) == -3
+    assert _cascade(lib, info_over={"plan_ints": 3}) == -3  # sizes that do not add up to the plan
+    assert _cascade(lib, info_over={"num_prefix_jobs": 99}) == -3
+    assert _cascade(lib, nb=0) == -3
+    assert _cascade(lib, qs=100) == -3
+    assert _cascade(lib, scale=float("inf")) == -3
+    assert _cascade(lib, q=None) == -1
+    assert _cascade(lib, plan=None) == -1
+    assert _cascade(lib, q=24) == -4
+    assert _cascade(lib, os_=516) == -4
+    assert _cascade(lib, ws=None) == -7
+    assert _cascade(lib, wsb=16) == -7
+    assert _cascade(lib, ws=264) == -7  # misaligned workspace
+    assert _cascade(lib, info_over={"num_seqs": 0, "plan_ints": 1, "num_jobs": 0, "num_members": 0,
+                                    "num_pieces": 0, "num_prefix_jobs": 0}) == 0
+    if not _has_gpu():  # never launch on the fake pointers used here
+        assert _cascade(lib) == -9
+
+
+def test_cascade_workspace_size_refuses_bad_input(lib):
+    plan = pa.cascade_plan(2, 4, 2, 16, 40)
+    assert pa.cascade_workspace_size(plan, 128) >= 256
+    assert pa.cascade_workspace_size(plan, 96) == 0
